@@ -1,0 +1,38 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module holds no attention arithmetic: it only draws q, k, v (and the upstream gradient dO) as iid
+N(0, 1) samples, multiplies them by ``sigma`` and rounds them to the requested dtype, in the
+``[batch, seqlen, nheads, headdim]`` layout of the skill page's ``flash_attn_func`` examples (page "Flash
+Attention — 長い系列を扱う Transformer の学習と推論を速くする", quick start and Workflow 2 Step 2).
+
+Recipe: one ``torch.Generator`` on the target device seeded with ``seed``; tensors drawn in the order
+q, k, v, dO as float32 ``randn``; each multiplied by ``sigma`` and then rounded (round-to-nearest-even) to
+fp16 or bf16. The rounded tensors are what both the CUDA path and the oracle consume.
+"""
+import torch
+
+DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def draw(shape, dtype, generator, device, sigma=1.0):
+    """One N(0,1)*sigma tensor drawn in float32, rounded to ``dtype``."""
+    x = torch.randn(shape, generator=generator, device=device, dtype=torch.float32)
+    if sigma != 1.0:
+        x.mul_(sigma)
+    return x.to(dtype)
+
+
+def make_inputs(B, Sq, Sk, H, D, dtype, seed, sigma=1.0, device="cuda", with_dout=False):
+    """q [B,Sq,H,D], k/v [B,Sk,H,D] (and dO [B,Sq,H,D]) drawn in that order from one seeded generator."""
+    if isinstance(dtype, str):
+        dtype = DTYPES[dtype]
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    q = draw((B, Sq, H, D), dtype, g, device, sigma)
+    k = draw((B, Sk, H, D), dtype, g, device, sigma)
+    v = draw((B, Sk, H, D), dtype, g, device, sigma)
+    if not with_dout:
+        return q, k, v
+    do = draw((B, Sq, H, D), dtype, g, device, 1.0)
+    return q, k, v, do
+

@@ -1,0 +1,267 @@
+"""Checks that pin the fp64 oracle to facts fixed outside itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` instance and raises AssertionError on a mismatch. The
+same functions run against the real oracle (tests/test_oracle_pins.py) and against copies of it with a
+planted mistake (tests/test_oracle_mutants.py), which must each fail at least one pin.
+
+What pins it:
+  * closed forms of special cases: a single key (O = v_0, LSE = s_00, dQ = dK = 0, dV_0 = sum_i dO_i);
+    identical keys (O_i = mean of the visible v_j, LSE_i = s + ln |J(i)|); the first causal row (O_0 = v_0);
+    V = ones gives O = 1 because every softmax row sums to 1;
+  * hand-worked examples with their derivations (tests/golden/hand_examples.json);
+  * invariants: joint permutation of (K, V) rows leaves a non-causal result unchanged; sum_j dK_j = 0 and
+    sum_j dV_j = sum_i dO_i per head;
+  * central finite differences of L = sum dO * O in fp64 on tiny shapes (the backward has no formula on
+    the pages, so the gradient of the oracle's own forward is the definition it must match);
+  * a library routine the definition reduces to: torch's scaled_dot_product_attention on the CPU in
+    float64, with autograd for the gradients (the skill page names SDPA in its quick start);
+  * the causal reading for Sq != Sk (bottom-right aligned) and fully masked rows (O = 0, LSE = -inf);
+  * the default scale 1/sqrt(d): the skill page divides by 8.0 for d = 64 (Workflow 1, Step 3 and 4).
+"""
+import json
+import math
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+TOL = 1e-12
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol * max(1.0, float(np.max(np.abs(b))) if b.size else 1.0), (what, err)
+
+
+def pin_single_key(orc):
+    r = _rng(1)
+    for causal in (False, True):
+        q = r.standard_normal((2, 5, 4)) if not causal else r.standard_normal((2, 1, 4))
+        k = r.standard_normal((2, 1, 4))
+        v = r.standard_normal((2, 1, 4))
+        do = r.standard_normal(q.shape)
+        out, lse = orc.fwd(q, k, v, causal=causal, scale=0.7)
+        Sq = q.shape[1]
+        _close(out, np.broadcast_to(v, (2, Sq, 4)), what="O = v0")
+        _close(lse, 0.7 * np.einsum("hid,hd->hi", q, k[:, 0]), what="LSE = s00")
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.7)
+        _close(dq, np.zeros_like(dq), what="dQ = 0")
+        _close(dk, np.zeros_like(dk), what="dK = 0")
+        _close(dv[:, 0], do.sum(axis=1), what="dV0 = sum dO")
+
+
+def pin_identical_keys(orc):
+    r = _rng(2)
+    S, D = 7, 3
+    q = r.standard_normal((1, S, D))
+    kk = r.standard_normal(D)
+    k = np.broadcast_to(kk, (1, S, D)).copy()
+    v = r.standard_normal((1, S, D))
+    out, lse = orc.fwd(q, k, v, causal=False, scale=0.3)
+    _close(out[0], np.broadcast_to(v[0].mean(axis=0), (S, D)), what="mean of V")
+    _close(lse[0], 0.3 * q[0] @ kk + math.log(S), what="LSE identical keys")
+    out, lse = orc.fwd(q, k, v, causal=True, scale=0.3)
+    for i in range(S):
+        _close(out[0, i], v[0, : i + 1].mean(axis=0), what="causal prefix mean")
+        _close(lse[0, i], 0.3 * q[0, i] @ kk + math.log(i + 1), what="causal LSE")
+
+
+def pin_first_causal_row(orc):
+    r = _rng(3)
+    q, k, v = (r.standard_normal((3, 6, 5)) for _ in range(3))
+    out, lse = orc.fwd(q, k, v, causal=True, scale=0.9, rows=np.zeros((3, 1), np.int64))
+    _close(out[:, 0], v[:, 0], what="O_0 = v_0")
+    _close(lse[:, 0], 0.9 * np.einsum("hd,hd->h", q[:, 0], k[:, 0]), what="LSE_0 = s_00")
+
+
+def pin_rows_sum_to_one(orc):
+    r = _rng(4)
+    for causal in (False, True):
+        q = r.standard_normal((2, 9, 4)) * 3
+        k = r.standard_normal((2, 9, 4)) * 3
+        v = np.ones((2, 9, 4))
+        out, _ = orc.fwd(q, k, v, causal=causal, scale=0.5)
+        _close(out, np.ones_like(out), tol=1e-14, what="softmax rows sum to 1")
+
+
+def pin_key_permutation(orc):
+    r = _rng(5)
+    q, k, v = (r.standard_normal((2, 8, 4)) for _ in range(3))
+    perm = r.permutation(8)
+    o1, l1 = orc.fwd(q, k, v, causal=False, scale=0.4)
+    o2, l2 = orc.fwd(q, k[:, perm], v[:, perm], causal=False, scale=0.4)
+    _close(o1, o2, what="perm O")
+    _close(l1, l2, what="perm LSE")
+
+
+def _loss(orc, q, k, v, do, causal, scale):
+    out, _ = orc.fwd(q, k, v, causal=causal, scale=scale)
+    return float(np.sum(out * do))
+
+
+def pin_finite_differences(orc):
+    r = _rng(6)
+    h = 1e-6
+    for (Sq, Sk, D, causal) in ((4, 4, 3, False), (5, 5, 2, True), (3, 6, 2, True), (6, 4, 3, True), (3, 5, 4, False)):
+        q = r.standard_normal((1, Sq, D))
+        k = r.standard_normal((1, Sk, D))
+        v = r.standard_normal((1, Sk, D))
+        do = r.standard_normal((1, Sq, D))
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.8)
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                xp = x.copy()
+                xp[idx] += h
+                xm = x.copy()
+                xm[idx] -= h
+                args_p = {"q": q, "k": k, "v": v}
+                args_m = dict(args_p)
+                args_p[name] = xp
+                args_m[name] = xm
+                num[idx] = (_loss(orc, args_p["q"], args_p["k"], args_p["v"], do, causal, 0.8)
+                            - _loss(orc, args_m["q"], args_m["k"], args_m["v"], do, causal, 0.8)) / (2 * h)
+            err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+            zero_ok = np.linalg.norm(num) < 1e-9 and np.linalg.norm(g) < 1e-9
+            assert zero_ok or err <= 1e-6, ("finite differences d" + name, Sq, Sk, causal, err)
+
+
+def pin_grad_invariants(orc):
+    r = _rng(7)
+    for causal in (False, True):
+        q, k, v, do = (r.standard_normal((2, 10, 4)) for _ in range(4))
+        _, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.6)
+        _close(dk.sum(axis=1), np.zeros((2, 4)), tol=1e-13, what="sum_j dK_j = 0")
+        _close(dv.sum(axis=1), do.sum(axis=1), tol=1e-13, what="sum_j dV_j = sum_i dO_i")
+
+
+def pin_row_subset(orc):
+    """dK/dV for a row subset equal the full gradient with dO zeroed outside the subset."""
+    r = _rng(8)
+    q, k, v, do = (r.standard_normal((2, 9, 3)) for _ in range(4))
+    rows = np.array([[0, 4, 8], [2, 3, 7]], np.int64)
+    dq_s, dk_s, dv_s = orc.bwd(q, k, v, do, causal=True, scale=0.5, rows=rows)
+    do_m = np.zeros_like(do)
+    for hh in range(2):
+        do_m[hh, rows[hh]] = do[hh, rows[hh]]
+    dq_f, dk_f, dv_f = orc.bwd(q, k, v, do_m, causal=True, scale=0.5)
+    _close(dk_s, dk_f, what="subset dK")
+    _close(dv_s, dv_f, what="subset dV")
+    for hh in range(2):
+        _close(dq_s[hh], dq_f[hh, rows[hh]], what="subset dQ")
+    o_s, l_s = orc.fwd(q, k, v, causal=True, scale=0.5, rows=rows)
+    o_f, l_f = orc.fwd(q, k, v, causal=True, scale=0.5)
+    for hh in range(2):
+        _close(o_s[hh], o_f[hh, rows[hh]], what="subset O")
+        _close(l_s[hh], l_f[hh, rows[hh]], what="subset LSE")
+
+
+def _sdpa(q, k, v, do, mask, scale):
+    import torch
+
+    tq = torch.tensor(q[None], dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(k[None], dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(v[None], dtype=torch.float64, requires_grad=True)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
+    o.backward(torch.tensor(do[None], dtype=torch.float64))
+    return (o.detach()[0].numpy(), tq.grad[0].numpy(), tk.grad[0].numpy(), tv.grad[0].numpy())
+
+
+def pin_sdpa_crosscheck(orc):
+    """float64 CPU SDPA ([B,H,S,D] after transposing; one batch of heads) with an explicit boolean mask."""
+    import torch
+
+    r = _rng(9)
+    for (Sq, Sk, D, causal) in ((16, 16, 8, False), (16, 16, 8, True), (5, 12, 4, True), (12, 12, 16, True),
+                                (7, 3, 4, False)):
+        H = 3
+        q = r.standard_normal((H, Sq, D))
+        k = r.standard_normal((H, Sk, D))
+        v = r.standard_normal((H, Sk, D))
+        do = r.standard_normal((H, Sq, D))
+        scale = 1.0 / math.sqrt(D)
+        mask = None
+        if causal:
+            # the bottom-right aligned reading, written as a boolean mask for SDPA
+            mask = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq)
+        o_ref, dq_ref, dk_ref, dv_ref = _sdpa(q, k, v, do, mask, scale)
+        out, lse = orc.fwd(q, k, v, causal=causal, scale=None)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=None)
+        _close(out, o_ref, what="SDPA O")
+        _close(dq, dq_ref, what="SDPA dQ")
+        _close(dk, dk_ref, what="SDPA dK")
+        _close(dv, dv_ref, what="SDPA dV")
+        # LSE against torch.logsumexp of the masked scores
+        s = torch.tensor(np.einsum("hid,hjd->hij", q, k) * scale)
+        if mask is not None:
+            s = s.masked_fill(~mask, float("-inf"))
+        _close(lse, torch.logsumexp(s, dim=-1).numpy(), what="logsumexp")
+
+
+def pin_causal_alignment(orc):
+    r = _rng(10)
+    # Sq < Sk: the last query sees every key, like the non-causal result; row i sees i + Sk - Sq + 1 keys.
+    q = r.standard_normal((1, 3, 4))
+    k = r.standard_normal((1, 7, 4))
+    v = r.standard_normal((1, 7, 4))
+    oc, lc = orc.fwd(q, k, v, causal=True, scale=0.5)
+    on, ln_ = orc.fwd(q, k, v, causal=False, scale=0.5)
+    _close(oc[0, 2], on[0, 2], what="last row sees all keys")
+    o5, l5 = orc.fwd(q[:, :1], k[:, :5], v[:, :5], causal=False, scale=0.5)
+    _close(oc[0, 0], o5[0, 0], what="row 0 sees keys 0..4")
+    _close(lc[0, 0], l5[0, 0], what="row 0 LSE")
+    # Sq > Sk: the first Sq - Sk rows see no key at all.
+    q = r.standard_normal((1, 6, 4))
+    k = r.standard_normal((1, 2, 4))
+    v = r.standard_normal((1, 2, 4))
+    do = r.standard_normal((1, 6, 4))
+    out, lse = orc.fwd(q, k, v, causal=True, scale=0.5)
+    assert np.all(out[0, :4] == 0.0) and np.all(np.isneginf(lse[0, :4])), "fully masked rows"
+    _close(out[0, 4], v[0, 0], what="first visible row sees key 0 only")
+    dq, dk, dv = orc.bwd(q, k, v, do, causal=True, scale=0.5)
+    assert np.all(dq[0, :4] == 0.0), "fully masked rows have zero dQ"
+
+
+def pin_default_scale(orc):
+    r = _rng(11)
+    q, k, v = (r.standard_normal((1, 4, 64)) for _ in range(3))
+    o_def, l_def = orc.fwd(q, k, v, scale=None)
+    o_8, l_8 = orc.fwd(q, k, v, scale=1.0 / 8.0)
+    _close(o_def, o_8, tol=0.0, what="default scale is 1/8 for d=64")
+    _close(l_def, l_8, tol=0.0, what="default scale LSE")
+
+
+def _parse(x):
+    if isinstance(x, list):
+        return [_parse(e) for e in x]
+    if isinstance(x, str):
+        coef, _, arg = x.partition("ln")
+        c = float(coef) if coef not in ("", "-") else (-1.0 if coef == "-" else 1.0)
+        return c * math.log(float(arg))
+    return float(x)
+
+
+def pin_golden_hand_examples(orc):
+    with open(os.path.join(HERE, "golden", "hand_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v, do = (np.array(_parse(c[n]))[None] for n in ("q", "k", "v", "dout"))
+        out, lse = orc.fwd(q, k, v, causal=c["causal"], scale=c["scale"])
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=c["causal"], scale=c["scale"])
+        _close(out[0], _parse(c["out"]), tol=1e-14, what=c["name"] + " O")
+        _close(lse[0], _parse(c["lse"]), tol=1e-14, what=c["name"] + " LSE")
+        _close(dq[0], _parse(c["dq"]), tol=1e-14, what=c["name"] + " dQ")
+        _close(dk[0], _parse(c["dk"]), tol=1e-14, what=c["name"] + " dK")
+        _close(dv[0], _parse(c["dv"]), tol=1e-14, what=c["name"] + " dV")
+
+
+ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
+            pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
+            pin_causal_alignment, pin_default_scale, pin_golden_hand_examples]

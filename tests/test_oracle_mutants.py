@@ -1,0 +1,58 @@
+"""Plant plausible mistakes in copies of the oracle source (on the CPU) and check that the pins catch each.
+
+Every mutant is a textual edit of oracle/fa_oracle.c compiled into a temporary directory: a dropped term, a
+wrong sign, a wrong index or operand, an off-by-one mask. The real oracle must pass every pin; each mutant
+must fail at least one.
+"""
+import os
+
+import pytest
+
+import oracle_pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "fa_oracle.c")
+
+MUTANTS = {
+    "drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "causal_off_by_one": ("return j <= i + (Sk - Sq);", "return j < i + (Sk - Sq);"),
+    "causal_top_left": ("return j <= i + (Sk - Sq);", "return j <= i;"),
+    "lse_drops_max": ("double lse = m + log(sum);", "double lse = log(sum);"),
+    "output_uses_k": ("o[d] += p[j] * vh[j * D + d];", "o[d] += p[j] * kh[j * D + d];"),
+    "dp_uses_k": ("acc += doh[i * D + d] * vh[j * D + d];", "acc += doh[i * D + d] * kh[j * D + d];"),
+    "ds_sign": ("dSi[j] = Pi[j] * (dP[j] - Di);", "dSi[j] = Pi[j] * (dP[j] + Di);"),
+    "drop_Di": ("Di += Pi[j] * dP[j];", "Di += 0.0 * dP[j];"),
+    "dq_no_scale": ("for (int64_t d = 0; d < D; ++d) dqi[d] *= scale;", ""),
+    "dq_uses_v": ("dqi[d] += dSi[j] * kh[j * D + d];", "dqi[d] += dSi[j] * vh[j * D + d];"),
+    "dk_uses_dout": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * doh[i * D + d];"),
+    "dv_uses_dS": ("gv += P[r * Sk + j] * doh[i * D + d];", "gv += dS[r * Sk + j] * doh[i * D + d];"),
+    "dk_no_scale": ("dkh[j * D + d] = scale * gk;", "dkh[j * D + d] = gk;"),
+    "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
+}
+
+
+@pytest.fixture(scope="module")
+def src_text():
+    with open(SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, src_text, tmp_path):
+    import oracle
+    from oracle import build as obuild
+
+    old, new = MUTANTS[name]
+    assert src_text.count(old) == 1, "mutation site not found exactly once: " + old
+    mutated = src_text.replace(old, new)
+    src = tmp_path / ("mutant_%s.c" % name)
+    src.write_text(mutated)
+    lib = obuild.build(str(src), str(tmp_path / ("libmutant_%s.so" % name)))
+    orc = oracle.Oracle(lib)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, "no pin caught the mutant " + name
