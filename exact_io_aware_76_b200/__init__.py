@@ -1,0 +1,136 @@
+"""B200-native (sm_100a) exact IO-aware attention: a thin Python binding over the C ABI of ``libfa.so``.
+
+Every step of the computation runs in the library's CUDA kernels; this module only marshals arguments
+(PyTorch tensors -> device pointers, sizes and the current CUDA stream) and turns status codes into
+exceptions. There is no fallback: if the library is missing or fails to load, every call raises.
+
+    fwd(q, k, v, causal=False, scale=None) -> (out, lse)
+    bwd(q, k, v, out, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
+
+Layouts follow the C header (include/fa.h): q/out/dout [B, Sq, H, D], k/v [B, Sk, H, D], fp16 or bf16,
+contiguous, on one CUDA device; lse is fp32 [B, H, Sq]. ``scale=None`` means 1/sqrt(D).
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa.so")
+
+FA_F16, FA_BF16 = 0, 1
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
+                -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status")
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (what, status_string(status), STATUS_NAMES.get(status, status)))
+
+
+def lib():
+    """The loaded ``libfa.so`` (ctypes.CDLL). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libfa.so not found at %s; build it with `python -m exact_io_aware_76_b200.build`"
+                          % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.restype = i
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+    L.fa_bwd.restype = i
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_status_string.argtypes = [i]
+    L.fa_device_status.restype = i
+    L.fa_device_status.argtypes = [i]
+    _lib = L
+    return L
+
+
+def status_string(status):
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.float16:
+        return FA_F16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    raise TypeError("expected float16 or bfloat16, got %s" % t.dtype)
+
+
+def _stream_ptr(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_bshd(name, t, dev):
+    if not t.is_cuda or t.device != dev:
+        raise ValueError("%s must be a CUDA tensor on %s" % (name, dev))
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous [B, S, H, D] tensor" % name)
+
+
+def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """Forward attention. Returns (out [B,Sq,H,D] in q's dtype, lse fp32 [B,H,Sq])."""
+    import torch
+
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_bshd(n, t, dev)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, D,
+                      int(bool(causal)), float(0.0 if scale is None else scale), _dtype_code(q), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd")
+    return out, lse
+
+
+def workspace_size(B, Sq, H, D):
+    return int(lib().fa_bwd_workspace_size(B, Sq, H, D))
+
+
+def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward attention (P recomputed from lse). Returns (dq, dk, dv) in q's dtype."""
+    import torch
+
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _check_bshd(n, t, dev)
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = workspace_size(B, Sq, H, D)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D, int(bool(causal)),
+                      float(0.0 if scale is None else scale), _dtype_code(q), workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def device_status(reset=False):
+    """The device-side sticky status word (FA_OK, or FA_ERR_TIMEOUT after a kernel gave up on a wait)."""
+    return int(lib().fa_device_status(int(bool(reset))))

@@ -1,0 +1,352 @@
+// fa_fwd.cuh -- forward exact attention for sm_100a: TMA-fed, mbarrier-pipelined, tcgen05 MMAs into TMEM,
+// warp-specialised online softmax.
+//
+// What it computes (page "Flash Attention — 長い系列を扱う Transformer の学習と推論を速くする", Workflow 1 Step 2,
+// and the glossary page "FlashAttention（フラッシュアテンション）とは？…", sections "FlashAttentionの仕組み" and
+// "Online Softmax"): O = softmax(scale * Q K^T + mask) V, split into tiles that are loaded on chip, with the
+// softmax normaliser updated as each key tile arrives, so the score matrix never reaches device memory.
+// Tile sizes follow the "64-128 rows x 64-128 columns" of page "FlashAttention-2 (2023)", section
+// "主な特徴・仕組み": 128 query rows x 128 keys, the natural M of a single-CTA tcgen05 MMA.
+//
+// Work unit: one CTA = (batch b, head h, 256 query rows = two 128-row Q tiles). Warp roles:
+//   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp 8     TMA producer: Q tiles once, then K/V tiles into a ring of kStages shared-memory stages
+//   warp 9     TMEM allocator and tcgen05 MMA issuer (one thread)
+//   warps 10-11 idle (they complete the third warpgroup, whose registers go to the softmax warpgroups)
+// Registers: 384 threads x 168 at launch; setmaxnreg moves the third warpgroup to 40 and the two softmax
+// warpgroups to 232 (2*128*232 + 128*40 = 64512 = 384*168), enough to hold a full 128-column S row.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D). P_t (16-bit) overwrites the
+// first 64 columns of S_t and is the A operand of the PV MMA read straight from TMEM.
+// The MMA issue order is S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ..., so while one warpgroup runs the
+// softmax of its tile the tensor core works on the other tile (ping-pong).
+//
+// Online softmax in the log2 domain: with c = scale*log2(e) and running max m (of s*c) and sum l,
+//   m' = max(m, rowmax(S)*c);  p = 2^(S*c - m');  l' = l*2^(m-m') + rowsum(p);  O' = O*2^(m-m') + P V.
+// The O rescale is lazy: m only moves when the new max exceeds it by more than kRescaleLog2 (8, i.e. a
+// factor 256); otherwise p is computed against the stale m. Both O and l use the same m, so the final
+// O/l is exact either way. LSE = (m + log2 l) * ln 2.
+#pragma once
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct FwdParams {
+  void* out;
+  float* lse;
+  int B, H, Sq, Sk;
+  int n_qblk;      // ceil(Sq / 256)
+  int n_kv_total;  // ceil(Sk / 128)
+  float scale_log2;  // scale * log2(e)
+};
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kBM = 128, kBN = 128, kNQ = 2;
+  static constexpr int kChunks = D / 64;              // 128-byte column chunks per row
+  static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile of 16-bit values
+  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kNQ * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B-swizzle atoms)
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegsSoftmax = 232, kRegsOther = 40;
+};
+
+template <int D, bool kBF16, bool kCausal>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + L::kStages;
+  uint64_t* kv_empty = v_full + L::kStages;
+  uint64_t* s_full = kv_empty + L::kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  // Heavy-first order for the causal mask: the last query blocks own the most key tiles.
+  const int bh = blockIdx.x % (p.B * p.H);
+  const int qblk_rank = blockIdx.x / (p.B * p.H);
+  const int qblk = kCausal ? (p.n_qblk - 1 - qblk_rank) : qblk_rank;
+  const int b = bh / p.H, h = bh % p.H;
+  const int off = p.Sk - p.Sq;  // bottom-right alignment of the causal mask
+
+  // Number of key tiles each Q tile visits (0: tile beyond Sq, or no visible key at all).
+  int n_kv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int row0 = qblk * 256 + t * 128;
+    if (row0 >= p.Sq) {
+      n_kv[t] = 0;
+    } else if (kCausal) {
+      const int last_row = min(p.Sq - 1, row0 + 127);
+      const int last_key = last_row + off;
+      n_kv[t] = last_key < 0 ? 0 : min(p.n_kv_total, last_key / 128 + 1);
+    } else {
+      n_kv[t] = p.n_kv_total;
+    }
+  }
+  const int n_iter = max(n_kv[0], n_kv[1]);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp >= 8) {
+    // setmaxnreg sits inside each role branch: ptxas rejects it ahead of a join shared by both kinds.
+    regs_dec<L::kRegsOther>();
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_iter > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      uint32_t q_bytes = 0;
+      for (int t = 0; t < 2; ++t) q_bytes += (n_kv[t] > 0) ? L::kTileBytes : 0;
+      mbar_arrive_expect_tx(q_full, q_bytes);
+      for (int t = 0; t < 2; ++t) {
+        if (n_kv[t] == 0) continue;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(smem + L::kQOff + t * L::kTileBytes + c * 16384, &tm_q, q_full, 64 * c, h,
+                      qblk * 256 + t * 128, b);
+      }
+      int j = 0;
+      for (; j < n_iter; ++j) {
+        const int s = j % L::kStages;
+        if (j >= L::kStages && !mbar_wait(&kv_empty[s], ((j / L::kStages) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(smem + L::kKOff + s * L::kTileBytes + c * 16384, &tm_k, &k_full[s], 64 * c, h, j * 128, b);
+        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(smem + L::kVOff + s * L::kTileBytes + c * 16384, &tm_v, &v_full[s], 64 * c, h, j * 128, b);
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA exits (bounded; own flag, not the CTA's).
+        int drain_flag = 0;
+        mbar_wait(q_full, 0, &drain_flag);
+        for (int jj = max(0, j - L::kStages); jj < j; ++jj) {
+          const int s = jj % L::kStages;
+          drain_flag = 0;
+          mbar_wait(&k_full[s], (jj / L::kStages) & 1, &drain_flag);
+          drain_flag = 0;
+          mbar_wait(&v_full[s], (jj / L::kStages) & 1, &drain_flag);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, D, false, true);
+      const uint32_t q_base = smem_u32(smem + L::kQOff);
+      const uint32_t k_base = smem_u32(smem + L::kKOff);
+      const uint32_t v_base = smem_u32(smem + L::kVOff);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      // S_t = Q_t K_j^T : K-major A and B, K (= head dim) advanced 16 elements (32 B) per instruction.
+      auto issue_qk = [&](int t, int s) {
+        const uint32_t s_tmem = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
+          const uint64_t a = sdesc_sw128(q_base + t * L::kTileBytes + koff, 16, 1024);
+          const uint64_t bd = sdesc_sw128(k_base + s * L::kTileBytes + koff, 16, 1024);
+          umma_ss(s_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V_j : A = P_t from TMEM (16 keys = 8 columns per instruction), B = V_j MN-major
+      // (16 keys = 16 rows of 128 B = 2048 B per instruction; 64-wide head-dim blocks 16 KB apart).
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t o_tmem = tmem + 256 + t * D;
+        const uint32_t p_tmem = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(v_base + s * L::kTileBytes + kk * 2048, 16384, 1024);
+          umma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        for (int t = 0; t < 2; ++t)
+          if (n_kv[t] > 0) {
+            issue_qk(t, 0);
+            umma_commit(&s_full[t]);
+          }
+      }
+      for (int j = 0; ok && j < n_iter; ++j) {
+        const int s = j % L::kStages;
+        const uint32_t ph = (j / L::kStages) & 1;
+        if (!mbar_wait(&v_full[s], ph, abort_flag)) break;
+        const int jn = j + 1;
+        bool next_k_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_kv[t]) continue;
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after_sync();
+          issue_pv(t, s, j > 0);
+          umma_commit(&o_full[t]);
+          if (jn < n_kv[t]) {
+            if (!next_k_ready) {
+              if (!mbar_wait(&k_full[jn % L::kStages], (jn / L::kStages) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after_sync();
+              next_k_ready = true;
+            }
+            issue_qk(t, jn % L::kStages);
+            umma_commit(&s_full[t]);
+          }
+        }
+        umma_commit(&kv_empty[s]);
+      }
+      // Every MMA must be complete before TMEM is released.
+      umma_commit(mma_done);
+      int drain_flag = 0;
+      mbar_wait(mma_done, 0, &drain_flag);
+    }
+  }
+  } else {
+    regs_inc<L::kRegsSoftmax>();
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp / 4;                 // Q tile of this warpgroup
+    const uint32_t quarter = warp % 4;      // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    const int row = qblk * 256 + t * 128 + row_in_tile;
+    const int nt = n_kv[t];
+    const uint32_t lane_base = tmem + ((quarter * 32) << 16);
+    const uint32_t s_tmem = lane_base + t * 128;
+    const uint32_t o_tmem = lane_base + 256 + t * D;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      if (!mbar_wait(&s_full[t], j & 1, abort_flag)) { ok = false; break; }
+      // PV(j-1) completed before S(j) (in-order tensor pipe); waiting keeps the o_full phases in step.
+      if (j > 0 && !mbar_wait(&o_full[t], (j - 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after_sync();
+      float s[128];
+      tmem_ld_x128(s_tmem, reinterpret_cast<uint32_t*>(s));
+      const int key0 = j * 128;
+      const bool need_mask = (key0 + 128 > p.Sk) || (kCausal && key0 + 127 > qblk * 256 + t * 128 + off);
+      if (need_mask) {
+        const int lim = kCausal ? min(p.Sk - 1, row + off) : (p.Sk - 1);  // last visible key of this row
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (key0 + c > lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = fmaxf(m, mx * p.scale_log2);
+      // Warp-uniform decision: TMEM loads/stores below are warp-collective.
+      const bool rescale = __any_sync(0xffffffffu, m_cand > m + kRescaleLog2);
+      if (rescale) {
+        const float alpha = ex2_approx(m - m_cand);  // 0 when m == -inf
+        if (j > 0) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
+            tmem_ld_x32(o_tmem + c0, reinterpret_cast<uint32_t*>(o));
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            tmem_st_x32(o_tmem + c0, reinterpret_cast<uint32_t*>(o));
+          }
+          tmem_st_wait();
+        }
+        l *= alpha;
+        m = m_cand;
+      }
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
+        const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
+        sum += p0 + p1;
+        pk[c / 2] = pack2<kBF16>(p0, p1);
+      }
+      l += sum;
+      tmem_st_x64(s_tmem, pk);
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(&p_full[t]);
+    }
+    // ---------------------------------------------------------------- epilogue: O / l and LSE
+    if (ok && nt > 0) ok = mbar_wait(&o_full[t], (nt - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after_sync();
+      const bool valid_row = row < p.Sq;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        if (nt > 0) {
+          tmem_ld_x32(o_tmem + c0, reinterpret_cast<uint32_t*>(o));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) w[c / 2] = pack2<kBF16>(o[c] * inv_l, o[c + 1] * inv_l);
+        if (valid_row) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (valid_row)
+        p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + row] = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,103 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention library, libfa.so.
+ *
+ * The operation (page "Flash Attention — 長い系列を扱う Transformer の学習と推論を速くする", quick start and
+ * Workflow 1 Step 2; page "FlashAttention（フラッシュアテンション）とは？…", sections "FlashAttentionの仕組み"
+ * and "Online Softmax"): exact scaled dot-product attention
+ *
+ *     O = softmax(scale * Q K^T + causal mask) V
+ *
+ * computed tile by tile with an online softmax, so the Sq x Sk score matrix never reaches device memory, plus
+ * the backward pass that recomputes the probabilities from the saved log-sum-exp ("tiling and recomputation",
+ * refbase entity page "FlashAttention", section "Capability"; training support: the glossary page's
+ * misconception 2).
+ *
+ * Conventions shared by every entry point
+ *   - Layout [batch, seqlen, nheads, headdim] ("[batch, seqlen, nheads, headdim]" in the skill page's
+ *     flash_attn_func examples), contiguous, row-major: element (b, s, h, d) sits at ((b*S + s)*H + h)*D + d.
+ *     q, out, dout, dq: [B, Sq, H, D];  k, v, dk, dv: [B, Sk, H, D];  lse: fp32 [B, H, Sq].
+ *   - dtype: FA_F16 or FA_BF16 for every 16-bit tensor of a call (the pages: fp16/bf16 only, no fp32).
+ *   - D (head dim) in {64, 128}. B, H, Sq, Sk >= 1. Every pointer 16-byte aligned, device memory.
+ *   - scale: 0.0f means 1/sqrt(D) (the pages' softmax_scale=None "Auto-scale"); any other finite value is
+ *     used as given.
+ *   - causal != 0 applies the causal mask, bottom-right aligned when Sq != Sk: key j is visible to query i
+ *     iff j <= i + (Sk - Sq). A query row that sees no key gets O = 0 and LSE = -inf.
+ *   - lse[b,h,i] = ln sum_{j visible} exp(scale * q_i . k_j), fp32 (natural log, scale included).
+ *   - Ownership: the caller allocates and owns every buffer, including the backward workspace. The library
+ *     allocates no device memory; it keeps no per-call state besides a device-side sticky error word.
+ *   - Asynchrony: all work is enqueued on `stream` (0 = legacy default stream). A return of FA_OK means the
+ *     launches were accepted, not that they finished. A kernel that gives up on an internal wait (bounded
+ *     spin, about 2 s) records FA_ERR_TIMEOUT in the device status word (fa_device_status) and exits cleanly.
+ *   - Errors: invalid arguments return FA_ERR_INVALID and launch nothing; an unsupported head dim, dtype or
+ *     device returns FA_ERR_UNSUPPORTED and launches nothing; a CUDA launch failure returns FA_ERR_CUDA.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t; /* identical to the CUDA runtime's definition */
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = -1,     /* bad pointer, size, alignment, scale or dtype; nothing launched */
+  FA_ERR_UNSUPPORTED = -2, /* head dim not in {64,128}, or the current device is not sm_100 */
+  FA_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed */
+  FA_ERR_TIMEOUT = -4,     /* device status only: a kernel gave up on a bounded wait */
+  FA_ERR_WORKSPACE = -5    /* backward workspace missing, misaligned or smaller than fa_bwd_workspace_size */
+} fa_status;
+
+/*
+ * Forward: out = softmax(scale * q k^T [+ mask]) v and lse (see conventions above).
+ *   q [B,Sq,H,D], k [B,Sk,H,D], v [B,Sk,H,D]: inputs, read only.
+ *   out [B,Sq,H,D]: written, same dtype as the inputs.  lse [B,H,Sq] fp32: written.
+ * Returns FA_OK or a negative fa_status.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H, int D,
+           int causal, float scale, int dtype, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes (0 on invalid sizes). The workspace holds the fp32
+ * dQ accumulator and the per-row fp32 terms D_i = rowsum(dO_i * O_i) and LSE_i * log2(e).
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int Sq, int H, int D);
+
+/*
+ * Backward: given the forward's inputs, its outputs out and lse, and the upstream gradient dout, writes
+ * dq [B,Sq,H,D], dk [B,Sk,H,D] and dv [B,Sk,H,D] (same dtype as the inputs). P is recomputed from lse; the S x S
+ * matrices never reach device memory.
+ *   workspace: caller-owned device buffer of at least fa_bwd_workspace_size(B,Sq,H,D) bytes, 256-byte aligned;
+ *              its contents on entry do not matter and are overwritten.
+ * Returns FA_OK or a negative fa_status (FA_ERR_WORKSPACE for a missing or short workspace).
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+           void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
+           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Static English description of a status code (never NULL). */
+FA_API const char* fa_status_string(int status);
+
+/*
+ * Device-side sticky status word of the current device: FA_OK, or FA_ERR_TIMEOUT once a kernel gave up on a
+ * bounded wait. Synchronises the device. With reset != 0 the word is cleared after reading. Returns the
+ * status, or FA_ERR_CUDA if it could not be read.
+ */
+FA_API int fa_device_status(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,97 @@
+"""Helpers shared by the GPU parity tests: move [B, S, H, D] tensors into the oracle's per-head fp64 layout,
+run the oracle on selected heads/rows, and apply the parity bounds.
+
+Parity bounds (the tolerance of the benchmark plan, with the reading for outputs the 16-bit format cannot
+represent that closely):
+  * O: |O - O_ref| <= tol * sigma + ulp(O_ref) / 2, tol = 1e-2 (bf16) or 2e-3 (fp16), sigma the input scale
+    (O is linear in V, so the bound scales with it), plus half a unit in the last place of the output format
+    at |O_ref| for the final rounding to 16 bits, which no implementation can avoid.
+  * LSE: |LSE - LSE_ref| <= 1e-3 where LSE_ref is finite; rows with no visible key must be -inf on both sides.
+  * dQ, dK, dV: ||G - G_ref||_F / ||G_ref||_F <= 2e-2 per tensor over the checked set.
+"""
+import numpy as np
+import torch
+
+import oracle
+
+O_TOL = {torch.bfloat16: 1e-2, torch.float16: 2e-3}
+LSE_TOL = 1e-3
+GRAD_RTOL = 2e-2
+MANT_BITS = {torch.bfloat16: 8, torch.float16: 11}  # significand bits incl. the implicit one
+
+
+def heads_f64(x, heads):
+    """x [B, S, H, D] (any device) -> float64 numpy [len(heads), S, D] for the (b, h) pairs in ``heads``."""
+    parts = [x[b, :, h, :].detach().to("cpu", torch.float64) for (b, h) in heads]
+    return torch.stack(parts).numpy()
+
+
+def all_heads(B, H):
+    return [(b, h) for b in range(B) for h in range(H)]
+
+
+def oracle_fwd(q, k, v, causal, scale, heads, rows=None):
+    return oracle.attn_fwd(heads_f64(q, heads), heads_f64(k, heads), heads_f64(v, heads), causal=causal,
+                           scale=scale, rows=rows)
+
+
+def oracle_bwd(q, k, v, do, causal, scale, heads, rows=None):
+    return oracle.attn_bwd(heads_f64(q, heads), heads_f64(k, heads), heads_f64(v, heads), heads_f64(do, heads),
+                           causal=causal, scale=scale, rows=rows)
+
+
+def gather_rows(x, heads, rows=None):
+    """x [B, S, H, D] -> float64 [n_heads, n_rows, D] (all rows if rows is None)."""
+    out = []
+    for t, (b, h) in enumerate(heads):
+        xs = x[b, :, h, :] if rows is None else x[b, torch.as_tensor(rows[t], device=x.device), h, :]
+        out.append(xs.detach().to("cpu", torch.float64))
+    return torch.stack(out).numpy()
+
+
+def gather_lse(lse, heads, rows=None):
+    out = []
+    for t, (b, h) in enumerate(heads):
+        ls = lse[b, h, :] if rows is None else lse[b, h, torch.as_tensor(rows[t], device=lse.device)]
+        out.append(ls.detach().to("cpu", torch.float64))
+    return torch.stack(out).numpy()
+
+
+def half_ulp(ref, dtype):
+    """Half a unit in the last place of ``dtype`` at |ref| (normal range)."""
+    a = np.maximum(np.abs(ref), 2.0 ** -14)
+    return 0.5 * 2.0 ** (np.floor(np.log2(a)) - (MANT_BITS[dtype] - 1))
+
+
+def check_out(o, o_ref, dtype, sigma=1.0, what="O"):
+    o = np.asarray(o, np.float64)
+    err = np.abs(o - o_ref)
+    bound = O_TOL[dtype] * sigma + half_ulp(o_ref, dtype)
+    bad = ~(err <= bound)
+    ulps = err / (2 * half_ulp(o_ref, dtype))
+    info = "%s: max err %.3e, max err/bound %.3f, max err %.2f ulp, %d/%d over" % (
+        what, float(err.max()) if err.size else 0.0, float((err / bound).max()) if err.size else 0.0,
+        float(ulps.max()) if ulps.size else 0.0, int(bad.sum()), err.size)
+    assert not bad.any(), info
+    return info
+
+
+def check_lse(lse, lse_ref, what="LSE"):
+    lse = np.asarray(lse, np.float64)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(lse), ~fin), what + ": -inf rows differ"
+    err = np.abs(lse[fin] - lse_ref[fin])
+    info = "%s: max err %.3e" % (what, float(err.max()) if err.size else 0.0)
+    assert err.size == 0 or err.max() <= LSE_TOL, info
+    return info
+
+
+def check_grad(g, g_ref, what):
+    g = np.asarray(g, np.float64)
+    num = np.linalg.norm(g - g_ref)
+    den = np.linalg.norm(g_ref)
+    rel = num / den if den > 0 else num
+    info = "%s: rel Frobenius err %.3e" % (what, rel)
+    assert np.all(np.isfinite(g)), what + ": non-finite values"
+    assert rel <= GRAD_RTOL, info
+    return info

@@ -1,0 +1,80 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the header declares,
+and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_76_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails first
+MISALIGNED = 0x10008
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    assert {"fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status"} <= names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(fa.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, 7):
+        s = fa.status_string(code)
+        assert isinstance(s, str) and s
+
+
+def fwd_call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Sq=128, Sk=128, H=1, D=64, causal=0, scale=0.0, dtype=0):
+    return fa.lib().fa_fwd(q, k, v, o, lse, B, Sq, Sk, H, D, causal, scale, dtype, None)
+
+
+@pytest.mark.parametrize("kw", [dict(q=None), dict(k=None), dict(v=None), dict(o=None), dict(lse=None),
+                                dict(q=MISALIGNED), dict(o=MISALIGNED), dict(lse=MISALIGNED), dict(B=0), dict(Sq=0),
+                                dict(Sk=-1), dict(H=0), dict(D=0), dict(scale=float("nan")),
+                                dict(scale=float("inf")), dict(scale=-0.5), dict(dtype=2)])
+def test_fwd_rejects_invalid(kw):
+    assert fwd_call(**kw) == -1
+
+
+@pytest.mark.parametrize("D", [32, 96, 256])
+def test_fwd_unsupported_head_dim(D):
+    assert fwd_call(D=D) == -2
+
+
+def bwd_call(ptr=FAKE, ws=FAKE, ws_bytes=1 << 30, B=1, Sq=128, Sk=128, H=1, D=64, scale=0.0, dtype=0, **over):
+    args = dict(q=ptr, k=ptr, v=ptr, o=ptr, lse=ptr, do=ptr, dq=ptr, dk=ptr, dv=ptr)
+    args.update(over)
+    return fa.lib().fa_bwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["do"], args["dq"],
+                           args["dk"], args["dv"], B, Sq, Sk, H, D, 1, scale, dtype, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw", [dict(q=None), dict(dq=None), dict(dk=MISALIGNED), dict(B=0), dict(scale=float("nan")),
+                                dict(dtype=5)])
+def test_bwd_rejects_invalid(kw):
+    assert bwd_call(**kw) == -1
+
+
+def test_bwd_workspace_checks():
+    need = fa.workspace_size(2, 300, 3, 64)
+    assert need > 0
+    assert bwd_call(B=2, Sq=300, H=3, ws=None) == -5
+    assert bwd_call(B=2, Sq=300, H=3, ws_bytes=need - 1) == -5
+    assert bwd_call(B=2, Sq=300, H=3, ws=FAKE + 16) == -5  # not 256-byte aligned
+
+
+def test_workspace_size_invalid_is_zero():
+    assert fa.workspace_size(0, 128, 1, 64) == 0
+    assert fa.workspace_size(1, 128, 1, 96) == 0

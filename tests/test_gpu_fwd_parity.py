@@ -1,0 +1,106 @@
+"""Forward parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Small workloads are compared element by element over every row; the GPT-style (4x32x8192x128) and long-context
+(1x32x131072x128) workloads on sampled rows (first row, last row, both sides of a tile edge, random rows),
+which the oracle computes one by one. Ragged and degenerate shapes cover partial tiles, Sq != Sk causal
+alignment, fully masked rows and single keys.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_76_b200 as fa
+from exact_io_aware_76_b200.inputs import make_inputs
+from exact_io_aware_76_b200.workloads import WORKLOADS, make_workload_inputs
+from parity_util import all_heads, check_lse, check_out, gather_lse, gather_rows, oracle_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_check(q, k, v, causal, scale, sigma, heads=None, rows=None, chunk=16):
+    """Run the CUDA forward once, then compare ``heads`` (rows ``rows``) with the oracle, ``chunk`` heads at a
+    time so that the fp64 host copies stay small."""
+    B, Sq, H, D = q.shape
+    out, lse = fa.fwd(q, k, v, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    heads = heads or all_heads(B, H)
+    info = []
+    for c0 in range(0, len(heads), chunk):
+        sub = heads[c0:c0 + chunk]
+        sub_rows = None if rows is None else rows[c0:c0 + chunk]
+        o_ref, l_ref = oracle_fwd(q, k, v, causal, scale, sub, sub_rows)
+        info.append(check_out(gather_rows(out, sub, sub_rows), o_ref, q.dtype, sigma))
+        info.append(check_lse(gather_lse(lse, sub, sub_rows), l_ref))
+    return info
+
+
+def sampled_rows(S, heads, per_head, seed):
+    """Rows 0 and S-1, both sides of the first 128-row tile edge, and random rows, per head."""
+    r = np.random.default_rng(seed)
+    base = [0, S - 1, min(127, S - 1), min(128, S - 1)]
+    rows = []
+    for _ in heads:
+        extra = r.choice(S, size=max(0, per_head - len(base)), replace=False)
+        rows.append(np.array((base + list(extra))[:per_head], dtype=np.int64))
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("name", ["tiny", "small_causal", "small_noncausal"])
+def test_small_workloads_full(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload_inputs(w)
+    print(run_and_check(q, k, v, w.causal, None, w.sigma))
+
+
+@pytest.mark.parametrize("name", sorted(n for n in WORKLOADS if n.startswith("mid_")))
+def test_mid_workloads(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload_inputs(w)
+    heads = [(0, 0), (0, 7), (1, 3), (1, 15)]  # full rows of 4 heads; every head's rows via the sampled test below
+    print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=heads))
+    hs = all_heads(w.B, w.H)
+    print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 6, 5)))
+
+
+@pytest.mark.parametrize("B,Sq,Sk,H,D,causal", [
+    (1, 1, 1, 1, 64, False), (1, 1, 1, 1, 128, True), (2, 300, 300, 3, 64, True), (2, 300, 300, 3, 128, False),
+    (1, 200, 333, 2, 64, True), (1, 333, 200, 2, 128, True), (1, 257, 129, 2, 64, False), (3, 130, 700, 5, 128, True),
+    (1, 5, 1000, 1, 64, True), (1, 1000, 5, 1, 128, True), (2, 511, 513, 2, 64, False), (1, 384, 384, 4, 128, True),
+])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_ragged_and_degenerate(B, Sq, Sk, H, D, causal, dtype):
+    q, k, v = make_inputs(B, Sq, Sk, H, D, dtype, seed=11 + Sq + 7 * Sk + D)
+    print(run_and_check(q, k, v, causal, None, 1.0))
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.3])
+def test_explicit_scale(scale):
+    q, k, v = make_inputs(1, 256, 256, 2, 64, "bf16", seed=3)
+    print(run_and_check(q, k, v, True, scale, 1.0))
+
+
+def test_single_key_closed_form():
+    """Sk = 1: every row's output is v_0 exactly and LSE is scale * q . k_0."""
+    q, k, v = make_inputs(2, 300, 1, 3, 128, "bf16", seed=21)
+    out, lse = fa.fwd(q, k, v, causal=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out, v.expand(2, 300, 3, 128))
+    ref = torch.einsum("bshd,bhd->bhs", q.double(), k[:, 0].double()) / math.sqrt(128)
+    assert (lse.double() - ref).abs().max().item() <= 1e-3
+
+
+def test_gpt_workload_sampled_rows():
+    w = WORKLOADS["gpt"]
+    q, k, v = make_workload_inputs(w)
+    hs = all_heads(w.B, w.H)
+    print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 4, 1)))
+
+
+def test_long_context_sampled_rows():
+    w = WORKLOADS["long"]
+    q, k, v = make_workload_inputs(w)
+    hs = all_heads(w.B, w.H)
+    print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 8, 2), chunk=4))

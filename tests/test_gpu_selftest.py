@@ -1,0 +1,50 @@
+"""tcgen05 / TMA layout self-checks on the GPU: one-CTA products through the test-only libfa_selftest.so, using
+the operand forms the attention kernels rely on, compared with a float32 product of the same 16-bit values."""
+import ctypes
+import os
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SELFTEST = os.path.join(ROOT, "exact_io_aware_76_b200", "libfa_selftest.so")
+
+VARIANTS = {0: "A K-major smem, B K-major smem", 1: "A K-major smem, B MN-major smem",
+            2: "A TMEM, B MN-major smem", 3: "A MN-major smem, B MN-major smem"}
+
+
+@pytest.fixture(scope="module")
+def st():
+    L = ctypes.CDLL(SELFTEST)
+    L.fa_selftest_umma.restype = ctypes.c_int
+    L.fa_selftest_umma.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                   ctypes.c_int, ctypes.c_int]
+    return L
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", sorted(VARIANTS))
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("K", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_umma_layouts(st, variant, N, K, dtype):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7 + variant * 100 + N + K)
+    if variant == 3:
+        a = torch.randn(K, 128, device="cuda", generator=g).to(dtype)  # stored [K][M]
+        a_mk = a.float().t()
+    else:
+        a = torch.randn(128, K, device="cuda", generator=g).to(dtype)
+        a_mk = a.float()
+    if variant == 0:
+        b = torch.randn(N, K, device="cuda", generator=g).to(dtype)  # stored [N][K]
+        b_kn = b.float().t()
+    else:
+        b = torch.randn(K, N, device="cuda", generator=g).to(dtype)  # stored [K][N]
+        b_kn = b.float()
+    c = torch.full((128, N), float("nan"), device="cuda", dtype=torch.float32)
+    rc = st.fa_selftest_umma(variant, a.data_ptr(), b.data_ptr(), c.data_ptr(), N, K, int(dtype == torch.bfloat16))
+    assert rc == 0, rc
+    ref = a_mk.double() @ b_kn.double()
+    err = (c.double() - ref).abs().max().item()
+    assert err <= 1e-3 * max(1.0, ref.abs().max().item()), (VARIANTS[variant], err)
