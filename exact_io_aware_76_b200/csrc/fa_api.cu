@@ -11,6 +11,8 @@
 
 namespace {
 
+using fa::BwdParams;
+using fa::BwdSmem;
 using fa::FwdParams;
 using fa::FwdSmem;
 
@@ -111,6 +113,57 @@ int dispatch_fwd_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& t
   return causal ? launch_fwd<D, BF16, true>(tq, tk, tv, p, dev, s) : launch_fwd<D, BF16, false>(tq, tk, tv, p, dev, s);
 }
 
+// ------------------------------------------------------------------------------------------------ backward
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+  size_t dq_acc, dvec, lse2, total;
+  int sq_pad;
+};
+
+// Workspace: fp32 dQ accumulator [B,H,Sq_pad,D], then D_i [B,H,Sq_pad], then LSE_i*log2(e) [B,H,Sq_pad].
+BwdLayout bwd_layout(int B, int Sq, int H, int D) {
+  BwdLayout l;
+  l.sq_pad = (Sq + 127) / 128 * 128;
+  const size_t rows = (size_t)B * H * l.sq_pad;
+  l.dq_acc = 0;
+  l.dvec = align256(rows * D * sizeof(float));
+  l.lse2 = l.dvec + align256(rows * sizeof(float));
+  l.total = l.lse2 + align256(rows * sizeof(float));
+  return l;
+}
+
+int grid_for(long long work, int per_block, int dev) {
+  long long g = (work + per_block - 1) / per_block;
+  const long long cap = (long long)g_dev[dev].sm_count * 8;
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+
+template <int D, bool BF16, bool CAUSAL>
+int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+               const BwdParams& p, int dev, cudaStream_t stream) {
+  static bool attr_done[kMaxDevices] = {};
+  auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL>;
+  int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
+  if (rc) return rc;
+  const long long rows = (long long)p.B * p.H * p.Sq_pad;
+  fa::fa_bwd_pre_kernel<D, BF16><<<grid_for(rows, 8, dev), 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  kern<<<(unsigned)(p.n_kblk * p.B * p.H), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;
+  fa::fa_bwd_dq_kernel<D, BF16><<<grid_for(n8, 256, dev), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int dispatch_bwd_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t s) {
+  return causal ? launch_bwd<D, BF16, true>(tq, tk, tv, tdo, p, dev, s)
+                : launch_bwd<D, BF16, false>(tq, tk, tv, tdo, p, dev, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -170,14 +223,57 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
                           : dispatch_fwd_causal<128, false>(c, tq, tk, tv, p, dev, stream);
 }
 
+size_t fa_bwd_workspace_size(int B, int Sq, int H, int D) {
+  if (check_common(B, Sq, 1, H, D, 1.f, FA_F16) != FA_OK) return 0;
+  return bwd_layout(B, Sq, H, D).total;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
+           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const void* ptrs[9] = {q, k, v, out, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return FA_ERR_INVALID;
+  int rc = check_common(B, Sq, Sk, H, D, scale, dtype);
+  if (rc) return rc;
+  const BwdLayout lay = bwd_layout(B, Sq, H, D);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < lay.total)
+    return FA_ERR_WORKSPACE;
+  int dev = 0;
+  if ((rc = current_device(&dev))) return rc;
+  if (scale == 0.f) scale = 1.f / sqrtf((float)D);
+
+  const int bq = (D == 128) ? BwdSmem<128>::kBQ : BwdSmem<64>::kBQ;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_bshd_map(&tq, q, B, Sq, H, D, dtype, bq))) return rc;
+  if ((rc = make_bshd_map(&tdo, dout, B, Sq, H, D, dtype, bq))) return rc;
+  if ((rc = make_bshd_map(&tk, k, B, Sk, H, D, dtype, 128))) return rc;
+  if ((rc = make_bshd_map(&tv, v, B, Sk, H, D, dtype, 128))) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdParams p;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq = dq;
+  p.dq_acc = reinterpret_cast<float*>(ws + lay.dq_acc);
+  p.dvec = reinterpret_cast<float*>(ws + lay.dvec);
+  p.lse2 = reinterpret_cast<float*>(ws + lay.lse2);
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.Sq_pad = lay.sq_pad;
+  p.n_kblk = (Sk + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  const bool c = causal != 0;
+  if (D == 64)
+    return dtype == FA_BF16 ? dispatch_bwd_causal<64, true>(c, tq, tk, tv, tdo, p, dev, stream)
+                            : dispatch_bwd_causal<64, false>(c, tq, tk, tv, tdo, p, dev, stream);
+  return dtype == FA_BF16 ? dispatch_bwd_causal<128, true>(c, tq, tk, tv, tdo, p, dev, stream)
+                          : dispatch_bwd_causal<128, false>(c, tq, tk, tv, tdo, p, dev, stream);
+}
+
 }  // extern "C"
-
-extern "C" size_t fa_bwd_workspace_size(int B, int Sq, int H, int D) {
-  (void)B; (void)Sq; (void)H; (void)D;
-  return 0;
-}
-
-extern "C" int fa_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
-                      void*, int, int, int, int, int, int, float, int, void*, size_t, cudaStream_t) {
-  return FA_ERR_UNSUPPORTED;
-}

@@ -1,3 +1,436 @@
-// fa_bwd.cuh -- backward kernels (placeholder until the recomputation backward lands).
+// fa_bwd.cuh -- recomputation backward of exact attention for sm_100a.
+//
+// The pages state that the method trains (forward and backward; glossary page "FlashAttention（フラッシュアテ
+// ンション）とは？…", misconception 2) and that it relies on tiling plus recomputation to keep memory linear in
+// the sequence length (refbase entity page "FlashAttention", section "Capability"). They give no backward
+// formulas; the ones below are the chain rule applied to O = softmax(scale * Q K^T + mask) V:
+//   P = exp(scale * S - LSE)            (recomputed from the saved LSE, never stored)
+//   dV = P^T dO,  dP = dO V^T,  D_i = rowsum(dO_i * O_i) = sum_j P_ij dP_ij,  dS = P * (dP - D)
+//   dQ = scale * dS K,  dK = scale * dS^T Q
+//
+// Three kernels, in stream order:
+//   fa_bwd_pre   D_i and LSE_i*log2(e) into the workspace (padded to a 128-row multiple), zero the fp32 dQ
+//                accumulator. HBM-bound elementwise work.
+//   fa_bwd_main  one CTA per (batch, head, 128-key tile); loops over the query tiles that see those keys.
+//   fa_bwd_dq    dQ = dtype(scale * dQacc), HBM-bound.
+//
+// fa_bwd_main warp roles:
+//   warps 0-3  "compute": thread = one key row (one TMEM lane). Reads S^T and dP^T rows from TMEM, forms
+//              P^T = 2^(S^T*c - LSE2) and dS^T = P^T (dP^T - D), writes P^T (16-bit) back to TMEM as the A
+//              operand of dV += P^T dO and dS^T (16-bit, 128-byte swizzled) to shared memory for the dK and dQ
+//              products; at the end writes dK (times scale) and dV.
+//   warps 4-7  "dQ": read each dQ partial out of TMEM and add it to the fp32 accumulator in global memory.
+//   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 2-stage ring.
+//   warp 9     TMEM allocator and tcgen05 MMA issuer.
+// Per query tile the MMAs are: S^T = K Q^T, dP^T = V dO^T (into TMEM), then dV += P^T dO (A from TMEM),
+// dK += dS^T Q, and dQ^T = K^T dS^T (D = 128; lane = head-dim index) or dQ = dS K (D = 64; lane = query),
+// the dQ partial landing in the dP^T columns that the compute warps have already consumed.
+// Query tile BQ = 64 rows for D = 128 and 128 rows for D = 64, so that every MMA has M = 128.
 #pragma once
 #include "sm100.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const void* out;   // [B,Sq,H,D]
+  const void* dout;  // [B,Sq,H,D]
+  const float* lse;  // [B,H,Sq]
+  void* dk;          // [B,Sk,H,D]
+  void* dv;          // [B,Sk,H,D]
+  void* dq;          // [B,Sq,H,D]
+  float* dq_acc;     // [B,H,Sq_pad,D] fp32
+  float* dvec;       // [B,H,Sq_pad]   D_i
+  float* lse2;       // [B,H,Sq_pad]   LSE_i * log2(e), +inf for padding rows and rows without keys
+  int B, H, Sq, Sk, Sq_pad;
+  int n_kblk;        // ceil(Sk / 128)
+  float scale, scale_log2;
+};
+
+constexpr float kLog2eB = 1.4426950408889634f;
+
+// ------------------------------------------------------------------------------------------ preprocess
+// One warp per (b, s, h) row: D = sum_d dO*O in fp32. Then zero dQacc with 16-byte stores.
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
+  const int warps_total = gridDim.x * 8;
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)p.B * p.H * p.Sq_pad;
+  constexpr int kPer = D / 32;  // elements per lane
+  for (long long r = gw; r < rows; r += warps_total) {
+    const int i = (int)(r % p.Sq_pad);
+    const long long bh = r / p.Sq_pad;
+    const int b = (int)(bh / p.H), h = (int)(bh % p.H);
+    float acc = 0.f;
+    if (i < p.Sq) {
+      const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.H + h) * D + lane * kPer;
+      const uint16_t* o = reinterpret_cast<const uint16_t*>(p.out) + base;
+      const uint16_t* g = reinterpret_cast<const uint16_t*>(p.dout) + base;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        float a, c;
+        if (kBF16) {
+          a = __uint_as_float(static_cast<uint32_t>(o[e]) << 16);
+          c = __uint_as_float(static_cast<uint32_t>(g[e]) << 16);
+        } else {
+          a = __half2float(__ushort_as_half(o[e]));
+          c = __half2float(__ushort_as_half(g[e]));
+        }
+        acc = fmaf(a, c, acc);
+      }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) {
+      float l2 = INFINITY;  // padding rows and rows that see no key: P = 2^(s - inf) = 0
+      if (i < p.Sq) {
+        const float l = p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + i];
+        if (l != -INFINITY) l2 = l * kLog2eB;
+      }
+      p.dvec[r] = (i < p.Sq) ? acc : 0.f;
+      p.lse2[r] = l2;
+    }
+  }
+  const long long n4 = (long long)p.B * p.H * p.Sq_pad * D / 4;
+  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n4; t += (long long)gridDim.x * blockDim.x)
+    acc4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ------------------------------------------------------------------------------------------ dQ convert
+template <int D, bool kBF16>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
+  const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;  // 8 outputs (16 bytes) per step
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n8; t += (long long)gridDim.x * blockDim.x) {
+    const long long e = t * 8;
+    const int d = (int)(e % D);
+    const long long row = e / D;  // (b*Sq + i)*H + h
+    const int h = (int)(row % p.H);
+    const long long bi = row / p.H;
+    const int i = (int)(bi % p.Sq), b = (int)(bi / p.Sq);
+    const float4* src =
+        reinterpret_cast<const float4*>(p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.Sq_pad + i) * D + d);
+    const float4 a = src[0], c = src[1];
+    uint4 w;
+    w.x = pack2<kBF16>(a.x * p.scale, a.y * p.scale);
+    w.y = pack2<kBF16>(a.z * p.scale, a.w * p.scale);
+    w.z = pack2<kBF16>(c.x * p.scale, c.y * p.scale);
+    w.w = pack2<kBF16>(c.z * p.scale, c.w * p.scale);
+    reinterpret_cast<uint4*>(p.dq)[t] = w;
+  }
+}
+
+// ------------------------------------------------------------------------------------------ main
+template <int D>
+struct BwdSmem {
+  static constexpr int kBQ = (D == 128) ? 64 : 128;  // query rows per iteration
+  static constexpr int kChunks = D / 64;
+  static constexpr int kKVBytes = 128 * D * 2;         // one 128-key tile of K or V
+  static constexpr int kQBytes = kBQ * D * 2;          // one query tile of Q or dO
+  static constexpr int kDSBytes = 128 * kBQ * 2;       // dS^T tile [128 keys][BQ queries]
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kKVBytes;
+  static constexpr int kQOff = kVOff + kKVBytes;          // 2 stages
+  static constexpr int kDOOff = kQOff + 2 * kQBytes;      // 2 stages
+  static constexpr int kDSOff = kDOOff + 2 * kQBytes;
+  static constexpr int kLOff = kDSOff + kDSBytes;         // LSE2, 2 stages x BQ floats
+  static constexpr int kDVecOff = kLOff + 2 * kBQ * 4;    // D_i, 2 stages x BQ floats
+  static constexpr int kBarOff = kDVecOff + 2 * kBQ * 4;
+  // kv_full, q_full[2], q_empty[2], sdp_full, ds_ready, dq_full, dq_empty, ds_empty, dkv_done
+  static constexpr int kNumBars = 11;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kAlloc = kMiscOff + 16 + 1024;
+  // TMEM columns: dV [0,D), dK [D,2D), S^T [2D, 2D+BQ), dP^T (and the dQ partial) [2D+BQ, 2D+2BQ)
+  static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + kBQ;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegsCompute = 240, kRegsOther = 40;
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D, bool kBF16, bool kCausal>
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr int BQ = L::kBQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;   // [2]
+  uint64_t* q_empty = bars + 3;  // [2]
+  uint64_t* sdp_full = bars + 5;
+  uint64_t* ds_ready = bars + 6;
+  uint64_t* dq_full = bars + 7;
+  uint64_t* dq_empty = bars + 8;
+  uint64_t* ds_empty = bars + 9;
+  uint64_t* dkv_done = bars + 10;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  // Heavy-first for the causal mask: the first key tiles are seen by the most query tiles.
+  const int bh = blockIdx.x % (p.B * p.H);
+  const int kblk = blockIdx.x / (p.B * p.H);
+  const int b = bh / p.H, h = bh % p.H;
+  const int off = p.Sk - p.Sq;
+  const int key0 = kblk * 128;
+  const int n_qtiles = (p.Sq + BQ - 1) / BQ;
+  int i_begin = 0;
+  if (kCausal) {
+    const int q_min = key0 - off;  // the first query that sees key0
+    i_begin = q_min <= 0 ? 0 : q_min / BQ;
+  }
+  const int n_it = max(0, n_qtiles - i_begin);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(sdp_full, 1);
+    mbar_init(ds_ready, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(ds_empty, 1);
+    mbar_init(dkv_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+  const size_t bh_row0 = static_cast<size_t>(bh) * p.Sq_pad;
+
+  if (warp >= 8) {
+    regs_dec<L::kRegsOther>();
+    if (warp == 8 && lane == 0 && n_it > 0) {
+      // ---------------------------------------------------------------- TMA producer
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kKVBytes);
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_4d(smem + L::kKOff + c * 16384, &tm_k, kv_full, 64 * c, h, key0, b);
+        tma_load_4d(smem + L::kVOff + c * 16384, &tm_v, kv_full, 64 * c, h, key0, b);
+      }
+      int it = 0;
+      for (; it < n_it; ++it) {
+        const int s = it & 1;
+        const int q0 = (i_begin + it) * BQ;
+        if (it >= 2 && !mbar_wait(&q_empty[s], ((it >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[s], 2 * L::kQBytes + 2 * BQ * 4);
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_4d(smem + L::kQOff + s * L::kQBytes + c * BQ * 128, &tm_q, &q_full[s], 64 * c, h, q0, b);
+          tma_load_4d(smem + L::kDOOff + s * L::kQBytes + c * BQ * 128, &tm_do, &q_full[s], 64 * c, h, q0, b);
+        }
+        bulk_load(smem + L::kLOff + s * BQ * 4, p.lse2 + bh_row0 + q0, BQ * 4, &q_full[s]);
+        bulk_load(smem + L::kDVecOff + s * BQ * 4, p.dvec + bh_row0 + q0, BQ * 4, &q_full[s]);
+      }
+      if (*abort_flag) {
+        int drain = 0;
+        mbar_wait(kv_full, 0, &drain);
+        for (int jj = max(0, it - 2); jj < it; ++jj) {
+          drain = 0;
+          mbar_wait(&q_full[jj & 1], (jj >> 1) & 1, &drain);
+        }
+      }
+    } else if (warp == 9 && lane == 0 && n_it > 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = idesc_f16(kBF16, 128, BQ, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_kv = idesc_f16(kBF16, 128, D, false, true);    // dV, dK
+      constexpr uint32_t idesc_q = (D == 128) ? idesc_f16(kBF16, 128, BQ, true, true)   // dQ^T = K^T dS^T
+                                              : idesc_f16(kBF16, 128, D, true, true);   // dQ = dS K
+      const uint32_t k_base = smem_u32(smem + L::kKOff), v_base = smem_u32(smem + L::kVOff);
+      const uint32_t q_base = smem_u32(smem + L::kQOff), do_base = smem_u32(smem + L::kDOOff);
+      const uint32_t ds_base = smem_u32(smem + L::kDSOff);
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&q_full[s], (it >> 1) & 1, abort_flag)) break;
+        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1, abort_flag)) break;
+        tc_fence_after_sync();
+        const uint32_t qs = q_base + s * L::kQBytes, dos = do_base + s * L::kQBytes;
+        // S^T = K Q^T and dP^T = V dO^T: K-major operands, head dim advanced 16 elements per instruction.
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
+          const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
+          umma_ss(tmem + L::kColS, sdesc_sw128(k_base + a_off, 16, 1024), sdesc_sw128(qs + b_off, 16, 1024), idesc_s,
+                  kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
+          const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
+          umma_ss(tmem + L::kColDP, sdesc_sw128(v_base + a_off, 16, 1024), sdesc_sw128(dos + b_off, 16, 1024),
+                  idesc_s, kk > 0);
+        }
+        umma_commit(sdp_full);
+        if (!mbar_wait(ds_ready, it & 1, abort_flag)) break;
+        tc_fence_after_sync();
+        // dV += P^T dO (A from TMEM) and dK += dS^T Q: the reduction runs over the BQ queries.
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint64_t bdo = sdesc_sw128(dos + kk * 2048, BQ * 128, 1024);
+          umma_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8, bdo, idesc_kv, (it > 0 || kk > 0));
+        }
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(ds_base + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bq = sdesc_sw128(qs + kk * 2048, BQ * 128, 1024);
+          umma_ss(tmem + L::kColDK, a, bq, idesc_kv, (it > 0 || kk > 0));
+        }
+        // dQ partial over this tile's 128 keys: MN-major operands, 16 keys (2048 B) per instruction.
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          uint64_t a, bd;
+          if (D == 128) {
+            a = sdesc_sw128(k_base + kk * 2048, 16384, 1024);   // K^T: M = head dim
+            bd = sdesc_sw128(ds_base + kk * 2048, 16384, 1024); // dS^T: N = queries
+          } else {
+            a = sdesc_sw128(ds_base + kk * 2048, 16384, 1024);  // dS: M = queries
+            bd = sdesc_sw128(k_base + kk * 2048, 16384, 1024);  // K: N = head dim
+          }
+          umma_ss(tmem + L::kColDP, a, bd, idesc_q, kk > 0);
+        }
+        umma_commit(dq_full);
+        umma_commit(ds_empty);
+        umma_commit(&q_empty[s]);
+      }
+      umma_commit(dkv_done);
+      int drain = 0;
+      mbar_wait(dkv_done, 0, &drain);
+    }
+  } else if (warp < 4) {
+    regs_inc<L::kRegsCompute>();
+    // ------------------------------------------------------------------ compute warpgroup (thread = key row)
+    const int j = warp * 32 + lane;   // key row within the tile = TMEM lane
+    const int key = key0 + j;
+    const uint32_t lane_base = tmem + ((warp * 32) << 16);
+    uint8_t* ds_row_base = smem + L::kDSOff + j * 128;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it & 1;
+      const int q0 = (i_begin + it) * BQ;
+      if (!mbar_wait(sdp_full, it & 1, abort_flag)) { ok = false; break; }
+      if (it > 0 && !mbar_wait(ds_empty, (it - 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after_sync();
+      const float* lse2 = reinterpret_cast<const float*>(smem + L::kLOff + s * BQ * 4);
+      const float* dvec = reinterpret_cast<const float*>(smem + L::kDVecOff + s * BQ * 4);
+      // Keys visible to query q satisfy key <= q + off, i.e. column c >= lo.
+      const int lo = kCausal ? (key - off - q0) : -1;
+      const bool need_mask = kCausal && (key0 + 127 > q0 + off);
+#pragma unroll
+      for (int c0 = 0; c0 < BQ; c0 += 32) {
+        float sv[32], dp[32];
+        tmem_ld_x32(lane_base + L::kColS + c0, reinterpret_cast<uint32_t*>(sv));
+        tmem_ld_x32(lane_base + L::kColDP + c0, reinterpret_cast<uint32_t*>(dp));
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -lse2[c0 + c]));
+          float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -lse2[c0 + c + 1]));
+          if (need_mask) {
+            if (c0 + c < lo) p0 = 0.f;
+            if (c0 + c + 1 < lo) p1 = 0.f;
+          }
+          const float d0 = p0 * (dp[c] - dvec[c0 + c]);
+          const float d1 = p1 * (dp[c + 1] - dvec[c0 + c + 1]);
+          pk[c / 2] = pack2<kBF16>(p0, p1);
+          dk[c / 2] = pack2<kBF16>(d0, d1);
+        }
+        tmem_st_x16(lane_base + L::kColS + c0 / 2, pk);
+        // dS^T row j, queries c0..c0+31 = four 16-byte units of the 128-byte swizzled row.
+        uint8_t* row = ds_row_base + (c0 / 64) * 16384;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = ((c0 % 64) / 8 + u) ^ (j & 7);
+          *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(ds_ready);
+    }
+    // ---------------------------------------------------------------- epilogue: dV and dK rows
+    if (ok && n_it > 0) ok = mbar_wait(dkv_done, 0, abort_flag);
+    if (ok) {
+      tc_fence_after_sync();
+      const bool valid = key < p.Sk;
+      const size_t row_off = ((static_cast<size_t>(b) * p.Sk + key) * p.H + h) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        uint16_t* dst = reinterpret_cast<uint16_t*>(which == 0 ? p.dv : p.dk) + row_off;
+        const float mul = which == 0 ? 1.f : p.scale;
+        const uint32_t col = which == 0 ? L::kColDV : L::kColDK;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          if (n_it > 0) {
+            tmem_ld_x32(lane_base + col + c0, reinterpret_cast<uint32_t*>(v));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = 0.f;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) w[c / 2] = pack2<kBF16>(v[c] * mul, v[c + 1] * mul);
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
+    const uint32_t quarter = warp - 4;
+    const int r = quarter * 32 + lane;  // TMEM lane: head-dim index (D = 128) or query row (D = 64)
+    const uint32_t lane_base = tmem + ((quarter * 32) << 16);
+    for (int it = 0; it < n_it; ++it) {
+      const int q0 = (i_begin + it) * BQ;
+      if (!mbar_wait(dq_full, it & 1, abort_flag)) break;
+      tc_fence_after_sync();
+      float v[64];
+      tmem_ld_x64(lane_base + L::kColDP, reinterpret_cast<uint32_t*>(v));
+      tc_fence_before_sync();
+      mbar_arrive(dq_empty);
+      if (D == 128) {
+        // lane r = head-dim index, column = query: 32 lanes add to 128 contiguous bytes per query.
+        float* base = p.dq_acc + (bh_row0 + q0) * D + r;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) atomicAdd(base + static_cast<size_t>(c) * D, v[c]);
+      } else {
+        // lane r = query row, column = head-dim index.
+        float* base = p.dq_acc + (bh_row0 + q0 + r) * D;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) red_add_v4(base + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -3,6 +3,7 @@
 // (TMEM allocation, MMA issue with shared-memory descriptors, commit to an mbarrier, TMEM loads/stores).
 #pragma once
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
