@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200: TFLOP/s of a GPT-style attention training step.
+
+A step is one pass of the whole path over one batch of synthetic input: the forward (O and LSE) and the
+recomputation backward (preprocess, main dK/dV/dQ kernel, dQ conversion) for B=4, H=32, Sq=Sk=8192, D=128,
+bf16, causal, with q, k, v and dO iid N(0,1) from a fixed seed. FLOPs: forward 4*B*H*D*pairs, backward
+10*B*H*D*pairs (five products, the recomputed Q K^T included), pairs = S(S+1)/2 visible (query, key) pairs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload gpt|long|...]
+
+Prints one JSON line (rank 0). ``value`` is the whole-job TFLOP/s from CUDA events with the inputs resident
+in HBM (1.07 GB per step, larger than the 126 MB L2); ``e2e`` is the same metric through the public Python API
+with pinned host inputs copied in and the gradients copied out every step; ``roofline`` rates the dominant
+kernel against the measured bf16 peak; ``cpu_baseline`` times the fp64 CPU oracle on a bounded row sample.
+With N > 1 (torchrun) every GPU runs its own replica of the workload (weak scaling, no collective on the data
+path) and the time is the maximum over ranks. ``--impl reference`` times the oracle itself as the reference
+arm (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+KERNEL_SOURCES = {
+    "fa_bwd_main": ["exact_io_aware_76_b200/csrc/fa_bwd.cuh", "exact_io_aware_76_b200/csrc/sm100.cuh"],
+    "fa_fwd": ["exact_io_aware_76_b200/csrc/fa_fwd.cuh", "exact_io_aware_76_b200/csrc/sm100.cuh"],
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gpt")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
+    ap.add_argument("--heads", type=int, default=None, help="override H (smaller cases for profiling)")
+    return ap.parse_args()
+
+
+def workload_from_args(args):
+    import dataclasses
+
+    from exact_io_aware_76_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.batch is not None or args.heads is not None:
+        B = args.batch or w.B
+        H = args.heads or w.H
+        w = dataclasses.replace(w, B=B, H=H, name="%s_b%dh%d" % (w.name, B, H))
+    return w
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("bf16_tflops", "bf16_tflops_sustained", "hbm_gbs")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(kernel):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)["%s/%s" % (kernel, workload)]
+    except Exception:
+        return None
+    if rec.get("source_sha") != source_sha(kernel):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of the SM clock, power and throttle reasons of one GPU."""
+
+    FIELDS = ["timestamp", "uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid):
+        self.uuid = (uuid or "").lower().replace("gpu-", "")
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.rows.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        def num(x):
+            try:
+                return float(x.split()[0])
+            except Exception:
+                return None
+
+        sel = []
+        for (ts, p) in self.rows:
+            if not (t0 <= ts <= t1 + 0.15):
+                continue
+            uid = p[1].lower().replace("gpu-", "")
+            if self.uuid and uid and uid != self.uuid:
+                continue
+            sel.append(p)
+        if not sel:
+            return None
+        sm = [num(p[2]) for p in sel if num(p[2]) is not None]
+        mx = [num(p[3]) for p in sel if num(p[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in sel for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sel),
+                "power_w_max": max((num(p[4]) for p in sel if num(p[4]) is not None), default=None)}
+
+
+# ------------------------------------------------------------------------------------------------ oracle leg
+def oracle_sample(w, q, k, v, do, seconds, seed=0):
+    """Time the fp64 oracle (forward + backward) on a bounded sample of query rows of one head of the workload.
+    Returns (TFLOP/s under the same FLOP convention, description, threads)."""
+    import numpy as np
+
+    import oracle
+
+    threads = len(os.sched_getaffinity(0))
+    to64 = lambda x: x[0, :, 0, :].detach().to("cpu").double().numpy()[None]  # noqa: E731
+    qh, kh, vh, doh = to64(q), to64(k), to64(v), to64(do)
+    rng = np.random.default_rng(seed)
+    fwd_only = w.name.startswith("long")
+
+    def flops(rows):
+        keys = np.minimum(w.Sk, rows + (w.Sk - w.Sq) + 1) if w.causal else np.full(rows.shape, w.Sk)
+        per = 4 if fwd_only else 14
+        return float(per * w.D * keys.sum())
+
+    def run(n):
+        rows = np.sort(rng.choice(w.Sq, n, replace=False)).astype(np.int64)[None]
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qh, kh, vh, causal=w.causal, rows=rows)
+        if not fwd_only:
+            oracle.attn_bwd(qh, kh, vh, doh, causal=w.causal, rows=rows)
+        return time.perf_counter() - t0, flops(rows[0])
+
+    dt, fl = run(8)  # calibration
+    n = int(min(w.Sq, max(8, 8 * seconds / max(dt, 1e-3))))
+    dt, fl = run(n)
+    desc = "%d random query rows of head (b=0,h=0) of the %s workload, %s, fp64 oracle" % (
+        n, w.name, "forward only" if fwd_only else "forward + backward")
+    return fl / dt / 1e12, desc, threads, dt
+
+
+# ------------------------------------------------------------------------------------------------ arms
+def run_reference(args):
+    from exact_io_aware_76_b200.inputs import make_inputs
+    from exact_io_aware_76_b200.replicas import env_rank
+
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    w = workload_from_args(args)
+    # One head of the workload's distribution is all the oracle sample reads (same recipe, generated on the CPU).
+    q, k, v, do = make_inputs(1, w.Sq, w.Sk, 1, w.D, w.dtype, w.seed, w.sigma, "cpu", with_dout=True)
+    per_step_s = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, do, per_step_s / 4)
+    vals, secs = [], 0.0
+    desc, threads = "", 0
+    for s in range(args.steps):
+        val, desc, threads, dt = oracle_sample(w, q, k, v, do, per_step_s / 4, seed=s + 1)
+        vals.append(val)
+        secs += dt
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": workload_config(w, 1),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, causal) and % of B200 dense tensor peak"
+
+
+def workload_config(w, n):
+    kind = "forward" if w.name.startswith("long") else "training step (forward + recomputation backward)"
+    return {"workload": "%s %s: B=%d H=%d Sq=%d Sk=%d D=%d %s %s" % (
+                w.name, kind, w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, "causal" if w.causal else "non-causal"),
+            "global_batch": w.B * n, "seq_len": w.Sq,
+            "parallelism": "replicas x%d (weak scaling; no collective on the data path)" % n,
+            "l2": "inputs larger than L2 (%.2f GB per step)" % (
+                (3 if w.name.startswith("long") else 4) * w.B * w.Sq * w.H * w.D * 2 / 1e9)}
+
+
+def run_ours(args):
+    import torch
+
+    import exact_io_aware_76_b200 as fa
+    from exact_io_aware_76_b200 import replicas
+    from exact_io_aware_76_b200.inputs import make_inputs
+
+    rank, world, local_rank = replicas.env_rank()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    replicas.init("nccl" if world > 1 else "gloo")
+    w = workload_from_args(args)
+    fwd_only = w.name.startswith("long")
+    seed = replicas.replica_seed(w.seed, rank)
+    q, k, v, do = make_inputs(w.B, w.Sq, w.Sk, w.H, w.D, w.dtype, seed, w.sigma, "cuda", with_dout=True)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.workspace_size(w.B, w.Sq, w.H, w.D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["fa_fwd"] if fwd_only else ["fa_fwd", "fa_bwd_pre", "fa_bwd_main", "fa_bwd_dq"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        fa.fwd(q, k, v, causal=w.causal, out=out, lse=lse)
+        mark(1)
+        if not fwd_only:
+            for st in range(3):
+                fa.bwd(q, k, v, out, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, stage=st)
+                mark(2 + st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0, "a kernel reported a timeout during warm-up"
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "")))
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.5)
+    replicas.barrier(dev)
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    replicas.barrier(dev)
+    local_ms = start.elapsed_time(stop)
+    max_ms = replicas.max_over_ranks(local_ms, dev)
+    if rank == 0:
+        sampler.stop()
+    status = fa.device_status()
+    assert status == 0, "a kernel reported status %d" % status
+
+    per_kernel = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                  for j, n in enumerate(names)}
+    flops_fwd = w.fwd_flops()
+    flops_bwd = 0 if fwd_only else w.bwd_flops()
+    flops_step = flops_fwd + flops_bwd
+    value = flops_step * world * K / (max_ms / 1e3) / 1e12
+
+    # ---- e2e through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv, hdo = (t.to("cpu").pin_memory() for t in (q, k, v, do))
+        outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ((out,) if fwd_only else (dq, dk, dv))]
+        h2d = sum(t.numel() * t.element_size() for t in ((hq, hk, hv) if fwd_only else (hq, hk, hv, hdo)))
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            if not fwd_only:
+                do.copy_(hdo, non_blocking=True)
+            o_, l_ = fa.fwd(q, k, v, causal=w.causal, out=out, lse=lse)
+            if fwd_only:
+                outs_h[0].copy_(o_, non_blocking=True)
+            else:
+                g = fa.bwd(q, k, v, o_, l_, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+                for hbuf, t in zip(outs_h, g):
+                    hbuf.copy_(t, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        replicas.barrier(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = replicas.max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": flops_step * world * args.e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    if rank != 0:
+        replicas.shutdown()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    dom = max(per_kernel, key=per_kernel.get)
+    dom_flops = flops_fwd if dom == "fa_fwd" else flops_bwd  # the backward's products all run in its main kernel
+    achieved = dom_flops / (per_kernel[dom] / 1e3) / 1e12
+    traffic = recorded_traffic(dom, w.name)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": "burst bf16 of %s" % peak_src,
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "frac_of_nominal_2250": achieved / NOMINAL_BF16_TFLOPS,
+                "algorithmic_flops_per_launch": dom_flops}
+    kernels = {n: {"ms": per_kernel[n]} for n in names}
+    kernels["fa_fwd"]["tflops"] = flops_fwd / (per_kernel["fa_fwd"] / 1e3) / 1e12
+    if not fwd_only:
+        kernels["fa_bwd_main"]["tflops"] = flops_bwd / (per_kernel["fa_bwd_main"] / 1e3) / 1e12
+        bwd_ms = per_kernel["fa_bwd_pre"] + per_kernel["fa_bwd_main"] + per_kernel["fa_bwd_dq"]
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        val, desc, threads, _ = oracle_sample(w, q, k, v, do, args.cpu_seconds)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+    clocks = sampler.summary(t_host0, t_host1)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world), "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(names) * K, "clocks": clocks,
+            "fwd_tflops": kernels["fa_fwd"]["tflops"],
+            "fwd_frac_of_measured_peak": kernels["fa_fwd"]["tflops"] / peaks["bf16_tflops"],
+            "kernels": kernels}
+    if not fwd_only:
+        line["bwd_tflops"] = flops_bwd / (bwd_ms / 1e3) / 1e12
+        line["bwd_frac_of_measured_peak"] = line["bwd_tflops"] / peaks["bf16_tflops"]
+        line["step_frac_of_measured_peak"] = (flops_step / ((per_kernel["fa_fwd"] + bwd_ms) / 1e3) / 1e12) / peaks["bf16_tflops"]
+    print(json.dumps(line), flush=True)
+    replicas.shutdown()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

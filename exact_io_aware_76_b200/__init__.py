@@ -20,7 +20,7 @@ FA_F16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
                 -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status")
+EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status")
 
 _lib = None
 
@@ -45,6 +45,8 @@ def lib():
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_bwd_stage.restype = i
+    L.fa_bwd_stage.argtypes = [i] + L.fa_bwd.argtypes
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_status_string.restype = ctypes.c_char_p
@@ -107,8 +109,12 @@ def workspace_size(B, Sq, H, D):
     return int(lib().fa_bwd_workspace_size(B, Sq, H, D))
 
 
-def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Backward attention (P recomputed from lse). Returns (dq, dk, dv) in q's dtype."""
+def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None,
+        stage=-1):
+    """Backward attention (P recomputed from lse). Returns (dq, dk, dv) in q's dtype.
+
+    ``stage`` selects one of the three launches (0 preprocess, 1 main, 2 dQ conversion; -1 all), see
+    ``fa_bwd_stage`` in include/fa.h; a caller running the stages separately must pass the same workspace."""
     import torch
 
     dev = q.device
@@ -122,10 +128,10 @@ def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=
     ws_bytes = workspace_size(B, Sq, H, D)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
-                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D, int(bool(causal)),
-                      float(0.0 if scale is None else scale), _dtype_code(q), workspace.data_ptr(),
-                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    rc = lib().fa_bwd_stage(int(stage), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D,
+                            int(bool(causal)), float(0.0 if scale is None else scale), _dtype_code(q),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
     return dq, dk, dv

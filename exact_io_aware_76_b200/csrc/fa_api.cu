@@ -140,28 +140,36 @@ int grid_for(long long work, int per_block, int dev) {
   return (int)(g < 1 ? 1 : g);
 }
 
+// stage -1: all three launches; 0: preprocess; 1: main; 2: dQ conversion.
 template <int D, bool BF16, bool CAUSAL>
-int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-               const BwdParams& p, int dev, cudaStream_t stream) {
+int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t stream) {
   static bool attr_done[kMaxDevices] = {};
   auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL>;
   int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
   if (rc) return rc;
-  const long long rows = (long long)p.B * p.H * p.Sq_pad;
-  fa::fa_bwd_pre_kernel<D, BF16><<<grid_for(rows, 8, dev), 256, 0, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  kern<<<(unsigned)(p.n_kblk * p.B * p.H), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;
-  fa::fa_bwd_dq_kernel<D, BF16><<<grid_for(n8, 256, dev), 256, 0, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (stage < 0 || stage == 0) {
+    const long long rows = (long long)p.B * p.H * p.Sq_pad;
+    fa::fa_bwd_pre_kernel<D, BF16><<<grid_for(rows, 8, dev), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (stage < 0 || stage == 1) {
+    kern<<<(unsigned)(p.n_kblk * p.B * p.H), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (stage < 0 || stage == 2) {
+    const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;
+    fa::fa_bwd_dq_kernel<D, BF16><<<grid_for(n8, 256, dev), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 template <int D, bool BF16>
-int dispatch_bwd_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int dispatch_bwd_causal(int stage, bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t s) {
-  return causal ? launch_bwd<D, BF16, true>(tq, tk, tv, tdo, p, dev, s)
-                : launch_bwd<D, BF16, false>(tq, tk, tv, tdo, p, dev, s);
+  return causal ? launch_bwd<D, BF16, true>(stage, tq, tk, tv, tdo, p, dev, s)
+                : launch_bwd<D, BF16, false>(stage, tq, tk, tv, tdo, p, dev, s);
 }
 
 }  // namespace
@@ -228,9 +236,10 @@ size_t fa_bwd_workspace_size(int B, int Sq, int H, int D) {
   return bwd_layout(B, Sq, H, D).total;
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout, void* dq,
-           void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
-           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal,
+                 float scale, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (stage < -1 || stage > 2) return FA_ERR_INVALID;
   const void* ptrs[9] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!ptr || !aligned16(ptr)) return FA_ERR_INVALID;
@@ -270,10 +279,17 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* out, const f
   p.scale_log2 = scale * fa::kLog2e;
   const bool c = causal != 0;
   if (D == 64)
-    return dtype == FA_BF16 ? dispatch_bwd_causal<64, true>(c, tq, tk, tv, tdo, p, dev, stream)
-                            : dispatch_bwd_causal<64, false>(c, tq, tk, tv, tdo, p, dev, stream);
-  return dtype == FA_BF16 ? dispatch_bwd_causal<128, true>(c, tq, tk, tv, tdo, p, dev, stream)
-                          : dispatch_bwd_causal<128, false>(c, tq, tk, tv, tdo, p, dev, stream);
+    return dtype == FA_BF16 ? dispatch_bwd_causal<64, true>(stage, c, tq, tk, tv, tdo, p, dev, stream)
+                            : dispatch_bwd_causal<64, false>(stage, c, tq, tk, tv, tdo, p, dev, stream);
+  return dtype == FA_BF16 ? dispatch_bwd_causal<128, true>(stage, c, tq, tk, tv, tdo, p, dev, stream)
+                          : dispatch_bwd_causal<128, false>(stage, c, tq, tk, tv, tdo, p, dev, stream);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout, void* dq,
+           void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
+           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return fa_bwd_stage(-1, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, D, causal, scale, dtype, workspace,
+                      workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -86,6 +86,19 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* out, 
            void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * The three launches of fa_bwd one at a time, for callers that time or schedule them separately:
+ *   stage 0: D_i = rowsum(dO_i * O_i) and LSE_i * log2(e) into the workspace, and zero its dQ accumulator;
+ *   stage 1: the main kernel (recomputes P per 128-key tile, writes dK and dV, accumulates dQ in fp32);
+ *   stage 2: dq = dtype(scale * dQ accumulator).
+ * Stages 0, 1, 2 in that order on one stream with identical arguments are exactly fa_bwd; stage -1 runs all
+ * three. Arguments, validation and return codes are those of fa_bwd (an unknown stage is FA_ERR_INVALID).
+ */
+FA_API int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D,
+                        int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
 /* Static English description of a status code (never NULL). */
 FA_API const char* fa_status_string(int status);
 
