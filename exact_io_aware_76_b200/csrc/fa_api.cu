@@ -293,3 +293,41 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* out, const f
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------ no-alloc
+// Backward for callers that cannot allocate device memory: the workspace is this fixed array in the
+// library's device image (see fa_bwd_noalloc in include/fa.h). Host code must not pass the array's name to
+// a kernel -- on the host it only stands in for the symbol -- so its device address is looked up once per
+// device with cudaGetSymbolAddress and cached.
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(int dev, void** ptr) {
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D,
+                              int causal, float scale, int dtype, cudaStream_t stream) {
+  int rc = check_common(B, Sq, Sk, H, D, scale, dtype);
+  if (rc) return rc;
+  if (fa_bwd_workspace_size(B, Sq, H, D) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  int dev = 0;
+  if ((rc = current_device(&dev))) return rc;
+  if (rc) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+  return fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, D, causal, scale, dtype, scratch,
+                FA_NOALLOC_SCRATCH_BYTES, stream);
+}

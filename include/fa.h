@@ -99,6 +99,32 @@ FA_API int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, 
                         int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+/*
+ * Size of the fixed device scratch that fa_bwd_noalloc uses in place of a caller workspace (64 MiB).
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * fa_bwd without a workspace argument and without any device allocation, for callers that cannot call
+ * cudaMalloc: for example a caller living inside another framework that owns every byte of device memory
+ * and forbids allocations outside its own pool, or a latency-critical caller that cannot afford the
+ * device-wide synchronisation cudaMalloc may cause. (The pages describe no such entry point; it is a
+ * convenience of this library.)
+ *   - The scratch is one statically sized array in the library's device image, FA_NOALLOC_SCRATCH_BYTES
+ *     long. Every GPU that loads the library holds it until the process exits.
+ *   - Problems whose fa_bwd_workspace_size exceeds FA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     FA_ERR_WORKSPACE before anything is launched (use fa_bwd with your own workspace for those).
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current; make that first call before any stream capture on the device.
+ *   - Every call shares the one array and it keeps the previous call's contents; the kernels clear what
+ *     must start at zero themselves. Calls whose kernels overlap on the GPU (two streams, or two host
+ *     threads) race on the array and give wrong gradients: serialise them.
+ * Other arguments, outputs and return codes are those of fa_bwd.
+ */
+FA_API int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D,
+                          int causal, float scale, int dtype, cudaStream_t stream);
+
 /* Static English description of a status code (never NULL). */
 FA_API const char* fa_status_string(int status);
 
