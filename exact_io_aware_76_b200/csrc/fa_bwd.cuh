@@ -19,8 +19,10 @@
 //              P^T = 2^(S^T*c - LSE2) and dS^T = P^T (dP^T - D), writes P^T (16-bit) back to TMEM as the A
 //              operand of dV += P^T dO and dS^T (16-bit, 128-byte swizzled) to shared memory for the dK and dQ
 //              products; at the end writes dK (times scale) and dV.
-//   warps 4-7  "dQ": read each dQ partial out of TMEM and add it to the fp32 accumulator in global memory.
-//   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 2-stage ring.
+//   warps 4-7  "dQ": read each dQ partial out of TMEM, stage it in shared memory and add it to the fp32
+//              accumulator in global memory with one bulk reduce-add per tile.
+//   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 3-stage (D=128) or 2-stage
+//              ring.
 //   warp 9     TMEM allocator and tcgen05 MMA issuer.
 // Per query tile the MMAs are: S^T = K Q^T, dP^T = V dO^T (into TMEM), then dV += P^T dO (A from TMEM),
 // dK += dS^T Q, and dQ^T = K^T dS^T (D = 128; lane = head-dim index) or dQ = dS K (D = 64; lane = query),
@@ -123,28 +125,34 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
 // ------------------------------------------------------------------------------------------ main
 template <int D>
 struct BwdSmem {
-  static constexpr int kBQ = (D == 128) ? 64 : 128;  // query rows per iteration
+  static constexpr int kBQ = (D == 128) ? 64 : 128;   // query rows per iteration
+  static constexpr int kNB = (D == 128) ? 2 : 1;      // S^T / dP^T / dS^T buffers (2 = pipelined)
+  static constexpr int kNQS = kNB + 1;                 // Q / dO / LSE2 / D stages
   static constexpr int kChunks = D / 64;
   static constexpr int kKVBytes = 128 * D * 2;         // one 128-key tile of K or V
   static constexpr int kQBytes = kBQ * D * 2;          // one query tile of Q or dO
   static constexpr int kDSBytes = 128 * kBQ * 2;       // dS^T tile [128 keys][BQ queries]
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKOff + kKVBytes;
-  static constexpr int kQOff = kVOff + kKVBytes;          // 2 stages
-  static constexpr int kDOOff = kQOff + 2 * kQBytes;      // 2 stages
-  static constexpr int kDSOff = kDOOff + 2 * kQBytes;
-  static constexpr int kLOff = kDSOff + kDSBytes;         // LSE2, 2 stages x BQ floats
-  static constexpr int kDVecOff = kLOff + 2 * kBQ * 4;    // D_i, 2 stages x BQ floats
-  static constexpr int kBarOff = kDVecOff + 2 * kBQ * 4;
-  // kv_full, q_full[2], q_empty[2], sdp_full, ds_ready, dq_full, dq_empty, ds_empty, dkv_done
-  static constexpr int kNumBars = 11;
+  static constexpr int kQOff = kVOff + kKVBytes;
+  static constexpr int kDOOff = kQOff + kNQS * kQBytes;
+  static constexpr int kDSOff = kDOOff + kNQS * kQBytes;
+  static constexpr int kDQBytes = kBQ * D * 4;            // fp32 dQ partial of one tile (32 KB)
+  static constexpr int kDQOff = kDSOff + kNB * kDSBytes;  // staging for the bulk reduction into dQacc
+  static constexpr int kLOff = kDQOff + kDQBytes;         // LSE2 per stage, BQ floats
+  static constexpr int kDVecOff = kLOff + kNQS * kBQ * 4;  // D_i per stage, BQ floats
+  static constexpr int kBarOff = kDVecOff + kNQS * kBQ * 4;
+  // kv_full, q_full[NQS], q_empty[NQS], sdp_full[NB], ds_ready[NB], dq_full[NB], dq_empty[NB], ds_empty[NB],
+  // dkv_done
+  static constexpr int kNumBars = 2 + 2 * kNQS + 5 * kNB;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
-  // TMEM columns: dV [0,D), dK [D,2D), S^T [2D, 2D+BQ), dP^T (and the dQ partial) [2D+BQ, 2D+2BQ)
-  static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + kBQ;
+  // TMEM columns: dV [0,D), dK [D,2D), S^T buffers from 2D, dP^T buffers (each also receives its tile's dQ
+  // partial once the compute warps have read dP^T) after them. D=128: 128+128+2*64+2*64 = 512 columns.
+  static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + kNB * kBQ;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
-  static constexpr uint32_t kRegsCompute = 240, kRegsOther = 40;
+  static constexpr uint32_t kRegsCompute = 232, kRegsOther = 64;  // dQ warpgroup keeps 168: 128*(232+168+64) <= 384*168
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -152,31 +160,36 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// Pipeline (NB = 2): the MMA thread issues S^T/dP^T of tile it+2 right after dV/dK/dQ of tile it, so the
+// compute warps work on tile it+1 while the tensor core runs both. Buffers are indexed by it % NB, stages
+// of the Q/dO ring by it % NQS; every barrier's phases are waited in order.
 template <int D, bool kBF16, bool kCausal>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const BwdParams p) {
   using L = BwdSmem<D>;
-  constexpr int BQ = L::kBQ;
+  constexpr int BQ = L::kBQ, NB = L::kNB, NQS = L::kNQS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;   // [2]
-  uint64_t* q_empty = bars + 3;  // [2]
-  uint64_t* sdp_full = bars + 5;
-  uint64_t* ds_ready = bars + 6;
-  uint64_t* dq_full = bars + 7;
-  uint64_t* dq_empty = bars + 8;
-  uint64_t* ds_empty = bars + 9;
-  uint64_t* dkv_done = bars + 10;
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = kv_full + 1;     // [NQS]
+  uint64_t* q_empty = q_full + NQS;   // [NQS]
+  uint64_t* sdp_full = q_empty + NQS; // [NB]
+  uint64_t* ds_ready = sdp_full + NB; // [NB]
+  uint64_t* dq_full = ds_ready + NB;  // [NB]
+  uint64_t* dq_empty = dq_full + NB;  // [NB]
+  uint64_t* ds_empty = dq_empty + NB; // [NB]
+  uint64_t* dkv_done = ds_empty + NB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
-  // Heavy-first for the causal mask: the first key tiles are seen by the most query tiles.
-  const int bh = blockIdx.x % (p.B * p.H);
-  const int kblk = blockIdx.x / (p.B * p.H);
+  // Head-major order: the key tiles of one (batch, head) run together, so its Q, dO and fp32 dQ accumulator
+  // stay resident in L2 while every key tile reads them and reduces into them; within a head, heavy-first
+  // for the causal mask (the first key tiles are seen by the most query tiles).
+  const int bh = blockIdx.x / p.n_kblk;
+  const int kblk = blockIdx.x % p.n_kblk;
   const int b = bh / p.H, h = bh % p.H;
   const int off = p.Sk - p.Sq;
   const int key0 = kblk * 128;
@@ -191,15 +204,17 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NQS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    mbar_init(sdp_full, 1);
-    mbar_init(ds_ready, 128);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_empty, 128);
-    mbar_init(ds_empty, 1);
+    for (int x = 0; x < NB; ++x) {
+      mbar_init(&sdp_full[x], 1);
+      mbar_init(&ds_ready[x], 128);
+      mbar_init(&dq_full[x], 1);
+      mbar_init(&dq_empty[x], 128);
+      mbar_init(&ds_empty[x], 1);
+    }
     mbar_init(dkv_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -229,9 +244,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       int it = 0;
       for (; it < n_it; ++it) {
-        const int s = it & 1;
+        const int s = it % NQS;
         const int q0 = (i_begin + it) * BQ;
-        if (it >= 2 && !mbar_wait(&q_empty[s], ((it >> 1) - 1) & 1, abort_flag)) break;
+        if (it >= NQS && !mbar_wait(&q_empty[s], ((it / NQS) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[s], 2 * L::kQBytes + 2 * BQ * 4);
         for (int c = 0; c < L::kChunks; ++c) {
           tma_load_4d(smem + L::kQOff + s * L::kQBytes + c * BQ * 128, &tm_q, &q_full[s], 64 * c, h, q0, b);
@@ -243,9 +258,9 @@ __global__ void __launch_bounds__(384, 1)
       if (*abort_flag) {
         int drain = 0;
         mbar_wait(kv_full, 0, &drain);
-        for (int jj = max(0, it - 2); jj < it; ++jj) {
+        for (int jj = max(0, it - NQS); jj < it; ++jj) {
           drain = 0;
-          mbar_wait(&q_full[jj & 1], (jj >> 1) & 1, &drain);
+          mbar_wait(&q_full[jj % NQS], (jj / NQS) & 1, &drain);
         }
       }
     } else if (warp == 9 && lane == 0 && n_it > 0) {
@@ -258,58 +273,68 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t q_base = smem_u32(smem + L::kQOff), do_base = smem_u32(smem + L::kDOOff);
       const uint32_t ds_base = smem_u32(smem + L::kDSOff);
       bool ok = mbar_wait(kv_full, 0, abort_flag);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(&q_full[s], (it >> 1) & 1, abort_flag)) break;
-        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1, abort_flag)) break;
+      // S^T = K Q^T and dP^T = V dO^T of tile `it` into buffer it % NB (K-major operands, head dim advanced
+      // 16 elements per instruction).
+      auto issue_sdp = [&](int it) -> bool {
+        const int x = it % NB, s = it % NQS;
+        if (!mbar_wait(&q_full[s], (it / NQS) & 1, abort_flag)) return false;
+        if (it >= NB && !mbar_wait(&dq_empty[x], ((it / NB) - 1) & 1, abort_flag)) return false;
         tc_fence_after_sync();
         const uint32_t qs = q_base + s * L::kQBytes, dos = do_base + s * L::kQBytes;
-        // S^T = K Q^T and dP^T = V dO^T: K-major operands, head dim advanced 16 elements per instruction.
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
-          umma_ss(tmem + L::kColS, sdesc_sw128(k_base + a_off, 16, 1024), sdesc_sw128(qs + b_off, 16, 1024), idesc_s,
-                  kk > 0);
+          umma_ss(tmem + L::kColS + x * BQ, sdesc_sw128(k_base + a_off, 16, 1024),
+                  sdesc_sw128(qs + b_off, 16, 1024), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
-          umma_ss(tmem + L::kColDP, sdesc_sw128(v_base + a_off, 16, 1024), sdesc_sw128(dos + b_off, 16, 1024),
-                  idesc_s, kk > 0);
+          umma_ss(tmem + L::kColDP + x * BQ, sdesc_sw128(v_base + a_off, 16, 1024),
+                  sdesc_sw128(dos + b_off, 16, 1024), idesc_s, kk > 0);
         }
-        umma_commit(sdp_full);
-        if (!mbar_wait(ds_ready, it & 1, abort_flag)) break;
+        umma_commit(&sdp_full[x]);
+        return true;
+      };
+      for (int it = 0; ok && it < min(NB, n_it); ++it) ok = issue_sdp(it);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int x = it % NB, s = it % NQS;
+        if (!mbar_wait(&ds_ready[x], (it / NB) & 1, abort_flag)) break;
         tc_fence_after_sync();
+        const uint32_t qs = q_base + s * L::kQBytes, dos = do_base + s * L::kQBytes;
+        const uint32_t dsb = ds_base + x * L::kDSBytes;
         // dV += P^T dO (A from TMEM) and dK += dS^T Q: the reduction runs over the BQ queries.
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint64_t bdo = sdesc_sw128(dos + kk * 2048, BQ * 128, 1024);
-          umma_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8, bdo, idesc_kv, (it > 0 || kk > 0));
+          umma_ts(tmem + L::kColDV, tmem + L::kColS + x * BQ + kk * 8, bdo, idesc_kv, (it > 0 || kk > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(ds_base + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t a = sdesc_sw128(dsb + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bq = sdesc_sw128(qs + kk * 2048, BQ * 128, 1024);
           umma_ss(tmem + L::kColDK, a, bq, idesc_kv, (it > 0 || kk > 0));
         }
-        // dQ partial over this tile's 128 keys: MN-major operands, 16 keys (2048 B) per instruction.
+        // dQ partial over this tile's 128 keys into the consumed dP^T buffer: MN-major operands, 16 keys
+        // (2048 B) per instruction.
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
           uint64_t a, bd;
           if (D == 128) {
             a = sdesc_sw128(k_base + kk * 2048, 16384, 1024);   // K^T: M = head dim
-            bd = sdesc_sw128(ds_base + kk * 2048, 16384, 1024); // dS^T: N = queries
+            bd = sdesc_sw128(dsb + kk * 2048, 16384, 1024);     // dS^T: N = queries
           } else {
-            a = sdesc_sw128(ds_base + kk * 2048, 16384, 1024);  // dS: M = queries
+            a = sdesc_sw128(dsb + kk * 2048, 16384, 1024);      // dS: M = queries
             bd = sdesc_sw128(k_base + kk * 2048, 16384, 1024);  // K: N = head dim
           }
-          umma_ss(tmem + L::kColDP, a, bd, idesc_q, kk > 0);
+          umma_ss(tmem + L::kColDP + x * BQ, a, bd, idesc_q, kk > 0);
         }
-        umma_commit(dq_full);
-        umma_commit(ds_empty);
+        umma_commit(&dq_full[x]);
+        umma_commit(&ds_empty[x]);
         umma_commit(&q_empty[s]);
+        if (it + NB < n_it && !issue_sdp(it + NB)) break;
       }
       umma_commit(dkv_done);
       int drain = 0;
@@ -321,51 +346,58 @@ __global__ void __launch_bounds__(384, 1)
     const int j = warp * 32 + lane;   // key row within the tile = TMEM lane
     const int key = key0 + j;
     const uint32_t lane_base = tmem + ((warp * 32) << 16);
-    uint8_t* ds_row_base = smem + L::kDSOff + j * 128;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int s = it & 1;
+      const int x = it % NB, s = it % NQS;
       const int q0 = (i_begin + it) * BQ;
-      if (!mbar_wait(sdp_full, it & 1, abort_flag)) { ok = false; break; }
-      if (it > 0 && !mbar_wait(ds_empty, (it - 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&sdp_full[x], (it / NB) & 1, abort_flag)) { ok = false; break; }
+      if (it >= NB && !mbar_wait(&ds_empty[x], ((it / NB) - 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after_sync();
       const float* lse2 = reinterpret_cast<const float*>(smem + L::kLOff + s * BQ * 4);
       const float* dvec = reinterpret_cast<const float*>(smem + L::kDVecOff + s * BQ * 4);
+      uint8_t* ds_row_base = smem + L::kDSOff + x * L::kDSBytes + j * 128;
+      const uint32_t s_col = L::kColS + x * BQ, dp_col = L::kColDP + x * BQ;
       // Keys visible to query q satisfy key <= q + off, i.e. column c >= lo.
       const int lo = kCausal ? (key - off - q0) : -1;
       const bool need_mask = kCausal && (key0 + 127 > q0 + off);
 #pragma unroll
-      for (int c0 = 0; c0 < BQ; c0 += 32) {
-        float sv[32], dp[32];
-        tmem_ld_x32(lane_base + L::kColS + c0, reinterpret_cast<uint32_t*>(sv));
-        tmem_ld_x32(lane_base + L::kColDP + c0, reinterpret_cast<uint32_t*>(dp));
-        uint32_t pk[16], dk[16];
+      for (int c0 = 0; c0 < BQ; c0 += 64) {
+        float sv[64], dp[64];
+        tmem_ld_x64_pair(lane_base + s_col + c0, reinterpret_cast<uint32_t*>(sv), lane_base + dp_col + c0,
+                         reinterpret_cast<uint32_t*>(dp));
+        uint32_t pk[32], dk[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -lse2[c0 + c]));
-          float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -lse2[c0 + c + 1]));
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
+          const float4 d4 = *reinterpret_cast<const float4*>(dvec + c0 + c);
+          float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -l4.x));
+          float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -l4.y));
+          float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l4.z));
+          float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l4.w));
           if (need_mask) {
             if (c0 + c < lo) p0 = 0.f;
             if (c0 + c + 1 < lo) p1 = 0.f;
+            if (c0 + c + 2 < lo) p2 = 0.f;
+            if (c0 + c + 3 < lo) p3 = 0.f;
           }
-          const float d0 = p0 * (dp[c] - dvec[c0 + c]);
-          const float d1 = p1 * (dp[c + 1] - dvec[c0 + c + 1]);
           pk[c / 2] = pack2<kBF16>(p0, p1);
-          dk[c / 2] = pack2<kBF16>(d0, d1);
+          pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+          dk[c / 2] = pack2<kBF16>(p0 * (dp[c] - d4.x), p1 * (dp[c + 1] - d4.y));
+          dk[c / 2 + 1] = pack2<kBF16>(p2 * (dp[c + 2] - d4.z), p3 * (dp[c + 3] - d4.w));
         }
-        tmem_st_x16(lane_base + L::kColS + c0 / 2, pk);
-        // dS^T row j, queries c0..c0+31 = four 16-byte units of the 128-byte swizzled row.
+        tmem_st_x32(lane_base + s_col + c0 / 2, pk);
+        // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
         uint8_t* row = ds_row_base + (c0 / 64) * 16384;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = ((c0 % 64) / 8 + u) ^ (j & 7);
+        for (int u = 0; u < 8; ++u) {
+          const int unit = u ^ (j & 7);
           *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(ds_ready);
+      mbar_arrive(&ds_ready[x]);
     }
     // ---------------------------------------------------------------- epilogue: dV and dK rows
     if (ok && n_it > 0) ok = mbar_wait(dkv_done, 0, abort_flag);
@@ -400,29 +432,47 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
+    // Each dQ partial goes TMEM -> registers -> a 32 KB fp32 staging tile in shared memory laid out exactly
+    // like the tile's rows of dQacc ([BQ][D], contiguous there), then one bulk reduce-add to global memory.
     const uint32_t quarter = warp - 4;
     const int r = quarter * 32 + lane;  // TMEM lane: head-dim index (D = 128) or query row (D = 64)
     const uint32_t lane_base = tmem + ((quarter * 32) << 16);
+    const bool leader = (warp == 4 && lane == 0);
+    float* stage = reinterpret_cast<float*>(smem + L::kDQOff);
     for (int it = 0; it < n_it; ++it) {
+      const int x = it % NB;
       const int q0 = (i_begin + it) * BQ;
-      if (!mbar_wait(dq_full, it & 1, abort_flag)) break;
+      // Uniform exit: all 128 threads leave together if any of them gave up on the wait.
+      if (!named_bar_and<1, 128>(mbar_wait(&dq_full[x], (it / NB) & 1, abort_flag))) break;
       tc_fence_after_sync();
       float v[64];
-      tmem_ld_x64(lane_base + L::kColDP, reinterpret_cast<uint32_t*>(v));
+      tmem_ld_x64(lane_base + L::kColDP + x * BQ, reinterpret_cast<uint32_t*>(v));
       tc_fence_before_sync();
-      mbar_arrive(dq_empty);
+      mbar_arrive(&dq_empty[x]);
+      if (it > 0) {
+        if (leader) bulk_wait_read_all();  // the previous reduction has read the staging tile
+        named_bar_sync<1, 128>();
+      }
       if (D == 128) {
-        // lane r = head-dim index, column = query: 32 lanes add to 128 contiguous bytes per query.
-        float* base = p.dq_acc + (bh_row0 + q0) * D + r;
+        // lane r = head-dim index, column = query: for each query the 32 lanes of a warp write 128 B.
 #pragma unroll
-        for (int c = 0; c < 64; ++c) atomicAdd(base + static_cast<size_t>(c) * D, v[c]);
+        for (int c = 0; c < 64; ++c) stage[c * D + r] = v[c];
       } else {
-        // lane r = query row, column = head-dim index.
-        float* base = p.dq_acc + (bh_row0 + q0 + r) * D;
+        // lane r = query row, column = head-dim index; rotate the 16-byte chunks to avoid bank conflicts.
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) red_add_v4(base + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+        for (int c = 0; c < 16; ++c) {
+          const int cc = (c + r) & 15;
+          *reinterpret_cast<float4*>(stage + r * D + cc * 4) = make_float4(v[4 * cc], v[4 * cc + 1], v[4 * cc + 2], v[4 * cc + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync<1, 128>();
+      if (leader) {
+        bulk_reduce_add_f32(p.dq_acc + (bh_row0 + q0) * D, stage, L::kDQBytes);
+        bulk_commit();
       }
     }
+    if (leader) bulk_wait_all();
   }
 
   tc_fence_before_sync();

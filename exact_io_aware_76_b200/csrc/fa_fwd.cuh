@@ -83,9 +83,11 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
-  // Heavy-first order for the causal mask: the last query blocks own the most key tiles.
-  const int bh = blockIdx.x % (p.B * p.H);
-  const int qblk_rank = blockIdx.x / (p.B * p.H);
+  // Head-major order: the query blocks of one (batch, head) run together, so its K and V stay resident in L2
+  // while they are re-read; within a head, heavy-first for the causal mask (the last query blocks own the
+  // most key tiles).
+  const int bh = blockIdx.x / p.n_qblk;
+  const int qblk_rank = blockIdx.x % p.n_qblk;
   const int qblk = kCausal ? (p.n_qblk - 1 - qblk_rank) : qblk_rank;
   const int b = bh / p.H, h = bh % p.H;
   const int off = p.Sk - p.Sq;  // bottom-right alignment of the causal mask
