@@ -17,6 +17,8 @@ using fa::FwdParams;
 using fa::FwdSmem;
 
 constexpr int kMaxDevices = 64;
+// Above this many bytes of re-read operands the kernels order CTAs head-major (about a third of the 126 MB L2).
+constexpr double kHeadMajorBytes = 48.0 * 1024 * 1024;
 
 // ------------------------------------------------------------------------------------------------ device
 struct DeviceInfo {
@@ -222,6 +224,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
   p.Sk = Sk;
   p.n_qblk = (Sq + 255) / 256;
   p.n_kv_total = (Sk + 127) / 128;
+  // Head-major CTA order once a head's re-read K/V no longer fit in L2 together with the other heads'.
+  p.head_major = (2.0 * B * Sk * H * D * 2 > kHeadMajorBytes) ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
   const bool c = causal != 0;
   if (D == 64)
@@ -275,6 +279,8 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
   p.Sk = Sk;
   p.Sq_pad = lay.sq_pad;
   p.n_kblk = (Sk + 127) / 128;
+  // Head-major CTA order once Q, dO and the fp32 dQ accumulator no longer fit in L2.
+  p.head_major = ((double)B * Sq * H * D * 8 > kHeadMajorBytes) ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * fa::kLog2e;
   const bool c = causal != 0;

@@ -16,11 +16,12 @@
 //
 // fa_bwd_main warp roles:
 //   warps 0-3  "compute": thread = one key row (one TMEM lane). Reads S^T and dP^T rows from TMEM, forms
-//              P^T = 2^(S^T*c - LSE2) and dS^T = P^T (dP^T - D), writes P^T (16-bit) back to TMEM as the A
-//              operand of dV += P^T dO and dS^T (16-bit, 128-byte swizzled) to shared memory for the dK and dQ
-//              products; at the end writes dK (times scale) and dV.
-//   warps 4-7  "dQ": read each dQ partial out of TMEM, stage it in shared memory and add it to the fp32
-//              accumulator in global memory with one bulk reduce-add per tile.
+//              P^T = 2^(S^T*c - LSE2) and dS^T = P^T (dP^T - D), writes both (16-bit) back to TMEM (over the
+//              S^T and dP^T columns it has read) as the A operands of dV += P^T dO and dK += dS^T Q, and dS^T
+//              (128-byte swizzled) to shared memory as an operand of the dQ product; at the end writes dK
+//              (times scale) and dV.
+//   warps 4-7  "dQ": read each dQ partial out of TMEM and add it to the fp32 accumulator in L2 with coalesced
+//              reductions straight from registers.
 //   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 3-stage (D=128) or 2-stage
 //              ring.
 //   warp 9     TMEM allocator and tcgen05 MMA issuer.
@@ -45,6 +46,7 @@ struct BwdParams {
   float* lse2;       // [B,H,Sq_pad]   LSE_i * log2(e), +inf for padding rows and rows without keys
   int B, H, Sq, Sk, Sq_pad;
   int n_kblk;        // ceil(Sk / 128)
+  int head_major;    // CTA order: 1 = all key tiles of a head together (L2 reuse), 0 = heavy-first
   float scale, scale_log2;
 };
 
@@ -137,9 +139,7 @@ struct BwdSmem {
   static constexpr int kQOff = kVOff + kKVBytes;
   static constexpr int kDOOff = kQOff + kNQS * kQBytes;
   static constexpr int kDSOff = kDOOff + kNQS * kQBytes;
-  static constexpr int kDQBytes = kBQ * D * 4;            // fp32 dQ partial of one tile (32 KB)
-  static constexpr int kDQOff = kDSOff + kNB * kDSBytes;  // staging for the bulk reduction into dQacc
-  static constexpr int kLOff = kDQOff + kDQBytes;         // LSE2 per stage, BQ floats
+  static constexpr int kLOff = kDSOff + kNB * kDSBytes;   // LSE2 per stage, BQ floats
   static constexpr int kDVecOff = kLOff + kNQS * kBQ * 4;  // D_i per stage, BQ floats
   static constexpr int kBarOff = kDVecOff + kNQS * kBQ * 4;
   // kv_full, q_full[NQS], q_empty[NQS], sdp_full[NB], ds_ready[NB], dq_full[NB], dq_empty[NB], ds_empty[NB],
@@ -152,7 +152,7 @@ struct BwdSmem {
   static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + kNB * kBQ;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
-  static constexpr uint32_t kRegsCompute = 232, kRegsOther = 64;  // dQ warpgroup keeps 168: 128*(232+168+64) <= 384*168
+  static constexpr uint32_t kRegsCompute = 216, kRegsDQ = 168, kRegsOther = 96;  // 128*(216+168+96) <= 384*168
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -185,11 +185,12 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
-  // Head-major order: the key tiles of one (batch, head) run together, so its Q, dO and fp32 dQ accumulator
-  // stay resident in L2 while every key tile reads them and reduces into them; within a head, heavy-first
-  // for the causal mask (the first key tiles are seen by the most query tiles).
-  const int bh = blockIdx.x / p.n_kblk;
-  const int kblk = blockIdx.x % p.n_kblk;
+  // CTA order. Head-major (large problems): the key tiles of one (batch, head) run together, so its Q, dO and
+  // fp32 dQ accumulator stay resident in L2 while every key tile reads them and reduces into them; heavy-first
+  // within the head (the first key tiles are seen by the most query tiles). Otherwise heavy-first across heads.
+  const int n_bh = p.B * p.H;
+  const int bh = p.head_major ? blockIdx.x / p.n_kblk : blockIdx.x % n_bh;
+  const int kblk = p.head_major ? blockIdx.x % p.n_kblk : blockIdx.x / n_bh;
   const int b = bh / p.H, h = bh % p.H;
   const int off = p.Sk - p.Sq;
   const int key0 = kblk * 128;
@@ -269,9 +270,16 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idesc_kv = idesc_f16(kBF16, 128, D, false, true);    // dV, dK
       constexpr uint32_t idesc_q = (D == 128) ? idesc_f16(kBF16, 128, BQ, true, true)   // dQ^T = K^T dS^T
                                               : idesc_f16(kBF16, 128, D, true, true);   // dQ = dS K
+      // Base descriptors are built once; every MMA adds a compile-time byte offset (plus a per-tile stage
+      // offset) to one of them, so the single issuing thread keeps up with the tensor core.
       const uint32_t k_base = smem_u32(smem + L::kKOff), v_base = smem_u32(smem + L::kVOff);
       const uint32_t q_base = smem_u32(smem + L::kQOff), do_base = smem_u32(smem + L::kDOOff);
       const uint32_t ds_base = smem_u32(smem + L::kDSOff);
+      const uint64_t k_kmaj = sdesc_sw128(k_base, 16, 1024), v_kmaj = sdesc_sw128(v_base, 16, 1024);
+      const uint64_t k_mn = sdesc_sw128(k_base, 16384, 1024);
+      const uint64_t q_kmaj = sdesc_sw128(q_base, 16, 1024), do_kmaj = sdesc_sw128(do_base, 16, 1024);
+      const uint64_t q_mn = sdesc_sw128(q_base, BQ * 128, 1024), do_mn = sdesc_sw128(do_base, BQ * 128, 1024);
+      const uint64_t ds_mn = sdesc_sw128(ds_base, 16384, 1024);
       bool ok = mbar_wait(kv_full, 0, abort_flag);
       // S^T = K Q^T and dP^T = V dO^T of tile `it` into buffer it % NB (K-major operands, head dim advanced
       // 16 elements per instruction).
@@ -280,20 +288,18 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&q_full[s], (it / NQS) & 1, abort_flag)) return false;
         if (it >= NB && !mbar_wait(&dq_empty[x], ((it / NB) - 1) & 1, abort_flag)) return false;
         tc_fence_after_sync();
-        const uint32_t qs = q_base + s * L::kQBytes, dos = do_base + s * L::kQBytes;
+        const uint64_t qd = sdesc_add(q_kmaj, s * L::kQBytes), dod = sdesc_add(do_kmaj, s * L::kQBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
-          umma_ss(tmem + L::kColS + x * BQ, sdesc_sw128(k_base + a_off, 16, 1024),
-                  sdesc_sw128(qs + b_off, 16, 1024), idesc_s, kk > 0);
+          umma_ss(tmem + L::kColS + x * BQ, sdesc_add(k_kmaj, a_off), sdesc_add(qd, b_off), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
-          umma_ss(tmem + L::kColDP + x * BQ, sdesc_sw128(v_base + a_off, 16, 1024),
-                  sdesc_sw128(dos + b_off, 16, 1024), idesc_s, kk > 0);
+          umma_ss(tmem + L::kColDP + x * BQ, sdesc_add(v_kmaj, a_off), sdesc_add(dod, b_off), idesc_s, kk > 0);
         }
         umma_commit(&sdp_full[x]);
         return true;
@@ -303,32 +309,23 @@ __global__ void __launch_bounds__(384, 1)
         const int x = it % NB, s = it % NQS;
         if (!mbar_wait(&ds_ready[x], (it / NB) & 1, abort_flag)) break;
         tc_fence_after_sync();
-        const uint32_t qs = q_base + s * L::kQBytes, dos = do_base + s * L::kQBytes;
-        const uint32_t dsb = ds_base + x * L::kDSBytes;
-        // dV += P^T dO (A from TMEM) and dK += dS^T Q: the reduction runs over the BQ queries.
+        const uint64_t qd = sdesc_add(q_mn, s * L::kQBytes), dod = sdesc_add(do_mn, s * L::kQBytes);
+        const uint64_t dsm = sdesc_add(ds_mn, x * L::kDSBytes);
+        // dV += P^T dO and dK += dS^T Q, both with A from TMEM: the reduction runs over the BQ queries.
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t bdo = sdesc_sw128(dos + kk * 2048, BQ * 128, 1024);
-          umma_ts(tmem + L::kColDV, tmem + L::kColS + x * BQ + kk * 8, bdo, idesc_kv, (it > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          umma_ts(tmem + L::kColDV, tmem + L::kColS + x * BQ + kk * 8, sdesc_add(dod, kk * 2048), idesc_kv,
+                  (it > 0 || kk > 0));
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(dsb + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
-          const uint64_t bq = sdesc_sw128(qs + kk * 2048, BQ * 128, 1024);
-          umma_ss(tmem + L::kColDK, a, bq, idesc_kv, (it > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          umma_ts(tmem + L::kColDK, tmem + L::kColDP + x * BQ + kk * 8, sdesc_add(qd, kk * 2048), idesc_kv,
+                  (it > 0 || kk > 0));
         // dQ partial over this tile's 128 keys into the consumed dP^T buffer: MN-major operands, 16 keys
-        // (2048 B) per instruction.
+        // (2048 B) per instruction. D = 128: dQ^T = K^T dS^T (M = head dim); D = 64: dQ = dS K (M = queries).
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
-          uint64_t a, bd;
-          if (D == 128) {
-            a = sdesc_sw128(k_base + kk * 2048, 16384, 1024);   // K^T: M = head dim
-            bd = sdesc_sw128(dsb + kk * 2048, 16384, 1024);     // dS^T: N = queries
-          } else {
-            a = sdesc_sw128(dsb + kk * 2048, 16384, 1024);      // dS: M = queries
-            bd = sdesc_sw128(k_base + kk * 2048, 16384, 1024);  // K: N = head dim
-          }
+          const uint64_t a = (D == 128) ? sdesc_add(k_mn, kk * 2048) : sdesc_add(dsm, kk * 2048);
+          const uint64_t bd = (D == 128) ? sdesc_add(dsm, kk * 2048) : sdesc_add(k_mn, kk * 2048);
           umma_ss(tmem + L::kColDP + x * BQ, a, bd, idesc_q, kk > 0);
         }
         umma_commit(&dq_full[x]);
@@ -386,6 +383,10 @@ __global__ void __launch_bounds__(384, 1)
           dk[c / 2 + 1] = pack2<kBF16>(p2 * (dp[c + 2] - d4.z), p3 * (dp[c + 3] - d4.w));
         }
         tmem_st_x32(lane_base + s_col + c0 / 2, pk);
+        // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
+        // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The tile's dQ partial lands on these columns
+        // later, issued after the dK product, and the tensor core executes in issue order.
+        tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
         // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
         uint8_t* row = ds_row_base + (c0 / 64) * 16384;
 #pragma unroll
@@ -432,47 +433,35 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else {
     // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
-    // Each dQ partial goes TMEM -> registers -> a 32 KB fp32 staging tile in shared memory laid out exactly
-    // like the tile's rows of dQacc ([BQ][D], contiguous there), then one bulk reduce-add to global memory.
+    // Each dQ partial goes TMEM -> registers -> fp32 reductions into dQacc in L2. (Staging it in shared memory
+    // for a bulk reduction costs 64 KB of shared-memory traffic per tile, which this kernel cannot spare: the
+    // MMAs' operand reads already come close to the shared-memory bandwidth.)
+    if constexpr (L::kRegsDQ < 168) regs_dec<L::kRegsDQ>();
     const uint32_t quarter = warp - 4;
     const int r = quarter * 32 + lane;  // TMEM lane: head-dim index (D = 128) or query row (D = 64)
     const uint32_t lane_base = tmem + ((quarter * 32) << 16);
-    const bool leader = (warp == 4 && lane == 0);
-    float* stage = reinterpret_cast<float*>(smem + L::kDQOff);
     for (int it = 0; it < n_it; ++it) {
       const int x = it % NB;
       const int q0 = (i_begin + it) * BQ;
-      // Uniform exit: all 128 threads leave together if any of them gave up on the wait.
-      if (!named_bar_and<1, 128>(mbar_wait(&dq_full[x], (it / NB) & 1, abort_flag))) break;
+      if (!mbar_wait(&dq_full[x], (it / NB) & 1, abort_flag)) break;
       tc_fence_after_sync();
       float v[64];
       tmem_ld_x64(lane_base + L::kColDP + x * BQ, reinterpret_cast<uint32_t*>(v));
       tc_fence_before_sync();
       mbar_arrive(&dq_empty[x]);
-      if (it > 0) {
-        if (leader) bulk_wait_read_all();  // the previous reduction has read the staging tile
-        named_bar_sync<1, 128>();
-      }
       if (D == 128) {
-        // lane r = head-dim index, column = query: for each query the 32 lanes of a warp write 128 B.
+        // lane r = head-dim index, column = query: for each query the 32 lanes of a warp add to 128 contiguous
+        // bytes (one coalesced reduction per query).
+        float* base = p.dq_acc + (bh_row0 + q0) * D + r;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) stage[c * D + r] = v[c];
+        for (int c = 0; c < 64; ++c) atomicAdd(base + static_cast<size_t>(c) * D, v[c]);
       } else {
-        // lane r = query row, column = head-dim index; rotate the 16-byte chunks to avoid bank conflicts.
+        // lane r = query row, column = head-dim index: 16-byte vector reductions along the row.
+        float* base = p.dq_acc + (bh_row0 + q0 + r) * D;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int cc = (c + r) & 15;
-          *reinterpret_cast<float4*>(stage + r * D + cc * 4) = make_float4(v[4 * cc], v[4 * cc + 1], v[4 * cc + 2], v[4 * cc + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync<1, 128>();
-      if (leader) {
-        bulk_reduce_add_f32(p.dq_acc + (bh_row0 + q0) * D, stage, L::kDQBytes);
-        bulk_commit();
+        for (int c = 0; c < 64; c += 4) red_add_v4(base + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
       }
     }
-    if (leader) bulk_wait_all();
   }
 
   tc_fence_before_sync();

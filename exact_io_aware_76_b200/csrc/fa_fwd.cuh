@@ -14,8 +14,8 @@
 //   warp 8     TMA producer: Q tiles once, then K/V tiles into a ring of kStages shared-memory stages
 //   warp 9     TMEM allocator and tcgen05 MMA issuer (one thread)
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go to the softmax warpgroups)
-// Registers: 384 threads x 168 at launch; setmaxnreg moves the third warpgroup to 40 and the two softmax
-// warpgroups to 232 (2*128*232 + 128*40 = 64512 = 384*168), enough to hold a full 128-column S row.
+// Registers: 384 threads x 168 at launch; setmaxnreg moves the third warpgroup to 88 and the two softmax
+// warpgroups to 208 (2*128*208 + 128*88 = 64512 = 384*168), enough to hold a full 128-column S row.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D). P_t (16-bit) overwrites the
 // first 64 columns of S_t and is the A operand of the PV MMA read straight from TMEM.
 // The MMA issue order is S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ..., so while one warpgroup runs the
@@ -41,6 +41,7 @@ struct FwdParams {
   int B, H, Sq, Sk;
   int n_qblk;      // ceil(Sq / 256)
   int n_kv_total;  // ceil(Sk / 128)
+  int head_major;  // CTA order: 1 = all query blocks of a head together (K/V reuse in L2), 0 = heavy-first
   float scale_log2;  // scale * log2(e)
 };
 
@@ -61,7 +62,7 @@ struct FwdSmem {
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B-swizzle atoms)
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
-  static constexpr uint32_t kRegsSoftmax = 232, kRegsOther = 40;
+  static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
 };
 
 template <int D, bool kBF16, bool kCausal>
@@ -83,11 +84,12 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
-  // Head-major order: the query blocks of one (batch, head) run together, so its K and V stay resident in L2
-  // while they are re-read; within a head, heavy-first for the causal mask (the last query blocks own the
-  // most key tiles).
-  const int bh = blockIdx.x / p.n_qblk;
-  const int qblk_rank = blockIdx.x % p.n_qblk;
+  // CTA order. Head-major (large problems): the query blocks of one (batch, head) run together, so its K and V
+  // stay resident in L2 while they are re-read, heavy-first within the head. Otherwise (everything fits in
+  // L2): heavy-first across all heads, which leaves the light blocks for the tail.
+  const int n_bh = p.B * p.H;
+  const int bh = p.head_major ? blockIdx.x / p.n_qblk : blockIdx.x % n_bh;
+  const int qblk_rank = p.head_major ? blockIdx.x % p.n_qblk : blockIdx.x / n_bh;
   const int qblk = kCausal ? (p.n_qblk - 1 - qblk_rank) : qblk_rank;
   const int b = bh / p.H, h = bh % p.H;
   const int off = p.Sk - p.Sq;  // bottom-right alignment of the causal mask
@@ -182,19 +184,20 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, D, false, true);
-      const uint32_t q_base = smem_u32(smem + L::kQOff);
-      const uint32_t k_base = smem_u32(smem + L::kKOff);
-      const uint32_t v_base = smem_u32(smem + L::kVOff);
+      // Base descriptors are built once; every MMA below adds a compile-time byte offset to one of them
+      // (building a descriptor per instruction would make this single issuing thread the bottleneck).
+      const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kVOff), 16384, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag);
       // S_t = Q_t K_j^T : K-major A and B, K (= head dim) advanced 16 elements (32 B) per instruction.
       auto issue_qk = [&](int t, int s) {
         const uint32_t s_tmem = tmem + t * 128;
+        const uint64_t a0 = sdesc_add(q_desc, t * L::kTileBytes), b0 = sdesc_add(k_desc, s * L::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-          const uint64_t a = sdesc_sw128(q_base + t * L::kTileBytes + koff, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_base + s * L::kTileBytes + koff, 16, 1024);
-          umma_ss(s_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss(s_tmem, sdesc_add(a0, koff), sdesc_add(b0, koff), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t V_j : A = P_t from TMEM (16 keys = 8 columns per instruction), B = V_j MN-major
@@ -202,11 +205,10 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_pv = [&](int t, int s, bool acc) {
         const uint32_t o_tmem = tmem + 256 + t * D;
         const uint32_t p_tmem = tmem + t * 128;
+        const uint64_t b0 = sdesc_add(v_desc, s * L::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_base + s * L::kTileBytes + kk * 2048, 16384, 1024);
-          umma_ts(o_tmem, p_tmem + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_ts(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * 2048), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {

@@ -74,21 +74,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of parity `parity` to complete. Returns false (and raises the CTA's abort flag
-// and the device status word) if the wait gave up, or if another thread of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// and the device status word) if the wait gave up after `limit_ns`, or if another thread of the CTA already
+// aborted.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t polls = 1;; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((polls & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (polls >= kWaitMaxPolls || globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (polls >= kWaitMaxPolls || globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicExch(&g_device_status, FA_ERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_ns(bar, parity, abort_flag, kWaitTimeoutNs);
 }
 
 // ---------------------------------------------------------------------------------------------------------
@@ -197,6 +202,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
+}
+
+// Advance a descriptor's start address by `bytes` (a multiple of 16). The address field holds addr >> 4 in its
+// low 14 bits and shared memory is below 256 KB, so a plain add never carries into the neighbouring fields;
+// with a compile-time `bytes` this is one integer add per MMA.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
 // Instruction descriptor, kind::f16, fp32 accumulator. is_bf16 selects bf16 (else fp16) for both A and B.

@@ -48,3 +48,27 @@ def test_umma_layouts(st, variant, N, K, dtype):
     ref = a_mk.double() @ b_kn.double()
     err = (c.double() - ref).abs().max().item()
     assert err <= 1e-3 * max(1.0, ref.abs().max().item()), (VARIANTS[variant], err)
+
+
+@pytest.mark.gpu
+def test_bounded_wait_gives_up_and_reports_timeout(st):
+    """A wait that nothing satisfies (an mbarrier no thread arrives on) must give up after its limit, record
+    FA_ERR_TIMEOUT in the device status word and return; the context stays usable afterwards."""
+    import time
+
+    import exact_io_aware_76_b200 as fa
+
+    st.fa_selftest_wait_timeout.restype = ctypes.c_int
+    st.fa_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_int)]
+    waited_ok = ctypes.c_int(-1)
+    t0 = time.perf_counter()
+    status = st.fa_selftest_wait_timeout(10_000_000, ctypes.byref(waited_ok))  # 10 ms limit
+    elapsed = time.perf_counter() - t0
+    assert status == -4, status
+    assert waited_ok.value == 0
+    assert elapsed < 5.0
+    # The GPU still works: a normal forward runs and the product library's status word is clean.
+    q = torch.randn(1, 128, 1, 64, device="cuda").half()
+    out, lse = fa.fwd(q, q, q)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and fa.device_status() == 0
