@@ -25,9 +25,9 @@
 //   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 3-stage (D=128) or 2-stage
 //              ring.
 //   warp 9     TMEM allocator and tcgen05 MMA issuer.
-// Per query tile the MMAs are: S^T = K Q^T, dP^T = V dO^T (into TMEM), then dV += P^T dO (A from TMEM),
-// dK += dS^T Q, and dQ^T = K^T dS^T (D = 128; lane = head-dim index) or dQ = dS K (D = 64; lane = query),
-// the dQ partial landing in the dP^T columns that the compute warps have already consumed.
+// Per query tile the MMAs are: dP^T = V dO^T, S^T = K Q^T (into TMEM), then dV += P^T dO and dK += dS^T Q
+// (A from TMEM), and dQ^T = K^T dS^T (D = 128; lane = head-dim index) or dQ = dS K (D = 64; lane = query),
+// the dQ partial landing in the S^T columns that the dV product has already read.
 // Query tile BQ = 64 rows for D = 128 and 128 rows for D = 64, so that every MMA has M = 128.
 #pragma once
 #include "sm100.cuh"
@@ -147,8 +147,8 @@ struct BwdSmem {
   static constexpr int kNumBars = 2 + 2 * kNQS + 5 * kNB;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
-  // TMEM columns: dV [0,D), dK [D,2D), S^T buffers from 2D, dP^T buffers (each also receives its tile's dQ
-  // partial once the compute warps have read dP^T) after them. D=128: 128+128+2*64+2*64 = 512 columns.
+  // TMEM columns: dV [0,D), dK [D,2D), S^T buffers from 2D (each later holds P^T and then its tile's dQ
+  // partial), dP^T buffers (later holding dS^T) after them. D=128: 128+128+2*64+2*64 = 512 columns.
   static constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColDP = 2 * D + kNB * kBQ;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
@@ -281,30 +281,38 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t q_mn = sdesc_sw128(q_base, BQ * 128, 1024), do_mn = sdesc_sw128(do_base, BQ * 128, 1024);
       const uint64_t ds_mn = sdesc_sw128(ds_base, 16384, 1024);
       bool ok = mbar_wait(kv_full, 0, abort_flag);
-      // S^T = K Q^T and dP^T = V dO^T of tile `it` into buffer it % NB (K-major operands, head dim advanced
-      // 16 elements per instruction).
-      auto issue_sdp = [&](int it) -> bool {
+      // dP^T = V dO^T and S^T = K Q^T of tile `it` into buffer it % NB (K-major operands, head dim advanced 16
+      // elements per instruction). dP^T first: its columns are free as soon as the previous tile of this
+      // buffer has been consumed, while the S^T columns also carry that tile's dQ partial, which the dQ warps
+      // must have read out first -- that wait then overlaps the dP^T products instead of emptying the pipe.
+      auto issue_dp = [&](int it) -> bool {
         const int x = it % NB, s = it % NQS;
         if (!mbar_wait(&q_full[s], (it / NQS) & 1, abort_flag)) return false;
-        if (it >= NB && !mbar_wait(&dq_empty[x], ((it / NB) - 1) & 1, abort_flag)) return false;
         tc_fence_after_sync();
-        const uint64_t qd = sdesc_add(q_kmaj, s * L::kQBytes), dod = sdesc_add(do_kmaj, s * L::kQBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
-          const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
-          umma_ss(tmem + L::kColS + x * BQ, sdesc_add(k_kmaj, a_off), sdesc_add(qd, b_off), idesc_s, kk > 0);
-        }
+        const uint64_t dod = sdesc_add(do_kmaj, s * L::kQBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
           const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
           umma_ss(tmem + L::kColDP + x * BQ, sdesc_add(v_kmaj, a_off), sdesc_add(dod, b_off), idesc_s, kk > 0);
         }
+        return true;
+      };
+      auto issue_s = [&](int it) -> bool {
+        const int x = it % NB, s = it % NQS;
+        if (it >= NB && !mbar_wait(&dq_empty[x], ((it / NB) - 1) & 1, abort_flag)) return false;
+        tc_fence_after_sync();
+        const uint64_t qd = sdesc_add(q_kmaj, s * L::kQBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a_off = (kk / 4) * 16384 + (kk % 4) * 32;
+          const uint32_t b_off = (kk / 4) * (BQ * 128) + (kk % 4) * 32;
+          umma_ss(tmem + L::kColS + x * BQ, sdesc_add(k_kmaj, a_off), sdesc_add(qd, b_off), idesc_s, kk > 0);
+        }
         umma_commit(&sdp_full[x]);
         return true;
       };
-      for (int it = 0; ok && it < min(NB, n_it); ++it) ok = issue_sdp(it);
+      for (int it = 0; ok && it < min(NB, n_it); ++it) ok = issue_dp(it) && issue_s(it);
       for (int it = 0; ok && it < n_it; ++it) {
         const int x = it % NB, s = it % NQS;
         if (!mbar_wait(&ds_ready[x], (it / NB) & 1, abort_flag)) break;
@@ -320,18 +328,19 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < BQ / 16; ++kk)
           umma_ts(tmem + L::kColDK, tmem + L::kColDP + x * BQ + kk * 8, sdesc_add(qd, kk * 2048), idesc_kv,
                   (it > 0 || kk > 0));
-        // dQ partial over this tile's 128 keys into the consumed dP^T buffer: MN-major operands, 16 keys
-        // (2048 B) per instruction. D = 128: dQ^T = K^T dS^T (M = head dim); D = 64: dQ = dS K (M = queries).
+        // dQ partial over this tile's 128 keys into the S^T columns (P^T there was read by the dV product,
+        // issued before): MN-major operands, 16 keys (2048 B) per instruction. D = 128: dQ^T = K^T dS^T
+        // (M = head dim); D = 64: dQ = dS K (M = queries).
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
           const uint64_t a = (D == 128) ? sdesc_add(k_mn, kk * 2048) : sdesc_add(dsm, kk * 2048);
           const uint64_t bd = (D == 128) ? sdesc_add(dsm, kk * 2048) : sdesc_add(k_mn, kk * 2048);
-          umma_ss(tmem + L::kColDP + x * BQ, a, bd, idesc_q, kk > 0);
+          umma_ss(tmem + L::kColS + x * BQ, a, bd, idesc_q, kk > 0);
         }
         umma_commit(&dq_full[x]);
         umma_commit(&ds_empty[x]);
         umma_commit(&q_empty[s]);
-        if (it + NB < n_it && !issue_sdp(it + NB)) break;
+        if (it + NB < n_it && !(issue_dp(it + NB) && issue_s(it + NB))) break;
       }
       umma_commit(dkv_done);
       int drain = 0;
@@ -384,7 +393,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         tmem_st_x32(lane_base + s_col + c0 / 2, pk);
         // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
-        // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The tile's dQ partial lands on these columns
+        // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The next tile's dP^T lands on these columns
         // later, issued after the dK product, and the tensor core executes in issue order.
         tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
         // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
@@ -446,7 +455,7 @@ __global__ void __launch_bounds__(384, 1)
       if (!mbar_wait(&dq_full[x], (it / NB) & 1, abort_flag)) break;
       tc_fence_after_sync();
       float v[64];
-      tmem_ld_x64(lane_base + L::kColDP + x * BQ, reinterpret_cast<uint32_t*>(v));
+      tmem_ld_x64(lane_base + L::kColS + x * BQ, reinterpret_cast<uint32_t*>(v));
       tc_fence_before_sync();
       mbar_arrive(&dq_empty[x]);
       if (D == 128) {
