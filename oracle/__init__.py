@@ -10,11 +10,13 @@ with the causal flag of the same page's quick start, and the chain-rule backward
 ``fa_oracle.c`` documents each step and the readings taken where the pages are silent.
 
 Array convention (numpy, float64, C-contiguous), one entry per attention head:
-    q, dout: [n_heads, Sq, D]      k, v: [n_heads, Sk, D]
-    rows:    [n_heads, n_rows] int64 query rows to evaluate (default: all rows)
+    q, dout: [n_q_heads, Sq, D]    k, v: [n_kv_heads, Sk, D]   (q head h reads K/V head h // (n_q / n_kv))
+    rows:    [n_q_heads, n_rows] int64 query rows to evaluate (default: all rows)
+    window:  (left, right) sliding window around the key aligned with each query; -1 = unbounded side
 Outputs:
-    fwd -> out [n_heads, n_rows, D], lse [n_heads, n_rows]   (natural-log LSE, scale included)
-    bwd -> dq [n_heads, n_rows, D], dk/dv [n_heads, Sk, D]   (dk/dv: contributions of the listed rows)
+    fwd -> out [n_q_heads, n_rows, D], lse [n_q_heads, n_rows]   (natural-log LSE, scale included)
+    bwd -> dq [n_q_heads, n_rows, D], dk/dv [n_kv_heads, Sk, D] (contributions of the listed rows, summed
+           over each group of q heads)
 
 Parity: pinned by tests/test_oracle_pins.py (closed forms, invariants, finite differences, hand-worked
 examples under tests/golden/, and a float64 PyTorch SDPA cross-check on tiny shapes).
@@ -45,13 +47,12 @@ class Oracle:
         self.libpath = libpath
         lib = ctypes.CDLL(libpath)
         lib.oracle_attn_fwd.restype = ctypes.c_int
-        lib.oracle_attn_fwd.argtypes = [_F64P, _F64P, _F64P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-                                        ctypes.c_int64, ctypes.c_int, ctypes.c_double, _I64P, ctypes.c_int64,
-                                        _F64P, _F64P]
+        i64 = ctypes.c_int64
+        lib.oracle_attn_fwd.argtypes = [_F64P, _F64P, _F64P, i64, i64, i64, i64, i64, ctypes.c_int, i64, i64,
+                                        ctypes.c_double, _I64P, i64, _F64P, _F64P]
         lib.oracle_attn_bwd.restype = ctypes.c_int
-        lib.oracle_attn_bwd.argtypes = [_F64P, _F64P, _F64P, _F64P, ctypes.c_int64, ctypes.c_int64,
-                                        ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_double, _I64P,
-                                        ctypes.c_int64, _F64P, _F64P, _F64P]
+        lib.oracle_attn_bwd.argtypes = [_F64P, _F64P, _F64P, _F64P, i64, i64, i64, i64, i64, ctypes.c_int, i64,
+                                        i64, ctypes.c_double, _I64P, i64, _F64P, _F64P, _F64P]
         self.lib = lib
 
     @staticmethod
@@ -59,8 +60,9 @@ class Oracle:
         q = np.ascontiguousarray(q, dtype=np.float64)
         k = np.ascontiguousarray(k, dtype=np.float64)
         v = np.ascontiguousarray(v, dtype=np.float64)
-        if q.ndim != 3 or k.ndim != 3 or v.shape != k.shape or q.shape[0] != k.shape[0] or q.shape[2] != k.shape[2]:
-            raise ValueError("expected q [n_heads,Sq,D], k/v [n_heads,Sk,D]")
+        if (q.ndim != 3 or k.ndim != 3 or v.shape != k.shape or q.shape[0] % k.shape[0] != 0
+                or q.shape[2] != k.shape[2]):
+            raise ValueError("expected q [n_q_heads,Sq,D], k/v [n_kv_heads,Sk,D] with n_kv_heads dividing n_q_heads")
         nh, Sq, D = q.shape
         if rows is None:
             rows = np.broadcast_to(np.arange(Sq, dtype=np.int64), (nh, Sq))
@@ -71,38 +73,40 @@ class Oracle:
             raise ValueError("rows must be [n_heads, n_rows]")
         return q, k, v, rows
 
-    def fwd(self, q, k, v, causal=False, scale=None, rows=None):
+    def fwd(self, q, k, v, causal=False, scale=None, rows=None, window=(-1, -1)):
         q, k, v, rows = self._prep(q, k, v, rows)
         nh, Sq, D = q.shape
-        Sk = k.shape[1]
+        nkv, Sk = k.shape[0], k.shape[1]
         if scale is None:
             scale = default_scale(D)
         nr = rows.shape[1]
         out = np.zeros((nh, nr, D), np.float64)
         lse = np.zeros((nh, nr), np.float64)
         rc = self.lib.oracle_attn_fwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P), v.ctypes.data_as(_F64P),
-                                      nh, Sq, Sk, D, int(bool(causal)), float(scale),
+                                      nh, nkv, Sq, Sk, D, int(bool(causal)), int(window[0]), int(window[1]),
+                                      float(scale),
                                       rows.ctypes.data_as(_I64P), nr, out.ctypes.data_as(_F64P),
                                       lse.ctypes.data_as(_F64P))
         if rc != 0:
             raise ValueError("oracle_attn_fwd rejected its arguments")
         return out, lse
 
-    def bwd(self, q, k, v, dout, causal=False, scale=None, rows=None):
+    def bwd(self, q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1)):
         q, k, v, rows = self._prep(q, k, v, rows)
         dout = np.ascontiguousarray(dout, dtype=np.float64)
         if dout.shape != q.shape:
             raise ValueError("dout must have q's shape")
         nh, Sq, D = q.shape
-        Sk = k.shape[1]
+        nkv, Sk = k.shape[0], k.shape[1]
         if scale is None:
             scale = default_scale(D)
         nr = rows.shape[1]
         dq = np.zeros((nh, nr, D), np.float64)
-        dk = np.zeros((nh, Sk, D), np.float64)
-        dv = np.zeros((nh, Sk, D), np.float64)
+        dk = np.zeros((nkv, Sk, D), np.float64)
+        dv = np.zeros((nkv, Sk, D), np.float64)
         rc = self.lib.oracle_attn_bwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P), v.ctypes.data_as(_F64P),
-                                      dout.ctypes.data_as(_F64P), nh, Sq, Sk, D, int(bool(causal)), float(scale),
+                                      dout.ctypes.data_as(_F64P), nh, nkv, Sq, Sk, D, int(bool(causal)),
+                                      int(window[0]), int(window[1]), float(scale),
                                       rows.ctypes.data_as(_I64P), nr, dq.ctypes.data_as(_F64P),
                                       dk.ctypes.data_as(_F64P), dv.ctypes.data_as(_F64P))
         if rc != 0:
@@ -120,14 +124,14 @@ def _get():
     return _default
 
 
-def attn_fwd(q, k, v, causal=False, scale=None, rows=None):
+def attn_fwd(q, k, v, causal=False, scale=None, rows=None, window=(-1, -1)):
     """O and LSE of the listed query rows (all rows by default). See the module docstring for layouts."""
-    return _get().fwd(q, k, v, causal=causal, scale=scale, rows=rows)
+    return _get().fwd(q, k, v, causal=causal, scale=scale, rows=rows, window=window)
 
 
-def attn_bwd(q, k, v, dout, causal=False, scale=None, rows=None):
+def attn_bwd(q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1)):
     """dQ of the listed rows and their dK/dV contributions. See the module docstring for layouts."""
-    return _get().bwd(q, k, v, dout, causal=causal, scale=scale, rows=rows)
+    return _get().bwd(q, k, v, dout, causal=causal, scale=scale, rows=rows, window=window)
 
 
 def bshd_heads(x, b, h):

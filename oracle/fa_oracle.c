@@ -15,18 +15,24 @@
  *      "FlashAttention（フラッシュアテンション）とは？…", section "よくある誤解", misconception 1.
  *  - Training (forward and backward) is supported; the pages give no backward formulas, so the backward
  *    here is the chain rule applied to the definition above.
+ *  - Multi-query / grouped-query attention ("K/V shared across heads", fewer KV heads) and sliding-window
+ *    attention (window_size = (left, right), (-1, -1) = none): skill page, Workflow 2, Steps 2 and 3.
  *
  * Readings where the pages are silent:
  *  - causal mask with Sq != Sk is bottom-right aligned: key j is visible to query i iff j <= i + (Sk - Sq);
+ *  - the window is aligned the same way: with c = i + (Sk - Sq), key j is visible iff
+ *    (left < 0 or j >= c - left) and (right < 0 or j <= c + right), on top of the causal condition;
+ *  - grouped heads: q head h reads K/V head h / (n_q_heads / n_kv_heads); dK and dV of a K/V head sum the
+ *    contributions of its group of q heads;
  *  - LSE_i is the natural log of sum_{j visible} exp(s_ij), scale included;
  *  - a query row with no visible key has O_i = 0, LSE_i = -inf and zero gradients.
  *
  * Layouts: every matrix is one attention head, row-major, fp64.
- *   q, dout : [n_heads][Sq][D]      k, v : [n_heads][Sk][D]
- *   rows    : [n_heads][n_rows]     query-row indices (0 <= rows < Sq) evaluated for each head
- *   out, dq : [n_heads][n_rows][D]  lse  : [n_heads][n_rows]
- *   dk, dv  : [n_heads][Sk][D]      contributions of the listed rows only (the gradient of
- *                                   L = sum over listed rows i of dout_i . O_i)
+ *   q, dout : [n_q_heads][Sq][D]      k, v : [n_kv_heads][Sk][D]   (n_q_heads a multiple of n_kv_heads)
+ *   rows    : [n_q_heads][n_rows]     query-row indices (0 <= rows < Sq) evaluated for each q head
+ *   out, dq : [n_q_heads][n_rows][D]  lse  : [n_q_heads][n_rows]
+ *   dk, dv  : [n_kv_heads][Sk][D]     contributions of the listed rows only (the gradient of
+ *                                     L = sum over listed rows i of dout_i . O_i), summed over each group
  * Return value: 0 on success, -1 on an invalid argument (nothing written).
  */
 #include <math.h>
@@ -34,11 +40,21 @@
 #include <stdlib.h>
 #include <string.h>
 
+/* The visibility rule of one problem: causal flag and window bounds (negative = unbounded). */
+struct mask {
+    int64_t Sq, Sk;
+    int causal;
+    int64_t left, right;
+};
+
 /* 1 if query row i may attend to key j. */
-static int visible(int64_t i, int64_t j, int64_t Sq, int64_t Sk, int causal)
+static int visible(int64_t i, int64_t j, const struct mask *m)
 {
-    if (!causal) return 1;
-    return j <= i + (Sk - Sq);
+    int64_t c = i + (m->Sk - m->Sq); /* the key aligned with query i */
+    if (m->causal && j > c) return 0;
+    if (m->left >= 0 && j < c - m->left) return 0;
+    if (m->right >= 0 && j > c + m->right) return 0;
+    return 1;
 }
 
 /* Scores s_ij = scale * q_i . k_j for one row, all keys. */
@@ -55,39 +71,42 @@ static void row_scores(const double *qi, const double *k, int64_t Sk, int64_t D,
  * Full (two-pass) softmax of one row over the visible keys. Writes p[j] = P_ij (0 where masked) and returns
  * LSE_i; returns -INFINITY and writes p = 0 when no key is visible.
  */
-static double row_softmax(const double *s, int64_t i, int64_t Sq, int64_t Sk, int causal, double *p)
+static double row_softmax(const double *s, int64_t i, const struct mask *mk, double *p)
 {
+    int64_t Sk = mk->Sk;
     double m = -INFINITY;
     for (int64_t j = 0; j < Sk; ++j)
-        if (visible(i, j, Sq, Sk, causal) && s[j] > m) m = s[j];
+        if (visible(i, j, mk) && s[j] > m) m = s[j];
     if (m == -INFINITY) {
         for (int64_t j = 0; j < Sk; ++j) p[j] = 0.0;
         return -INFINITY;
     }
     double sum = 0.0;
     for (int64_t j = 0; j < Sk; ++j)
-        if (visible(i, j, Sq, Sk, causal)) sum += exp(s[j] - m);
+        if (visible(i, j, mk)) sum += exp(s[j] - m);
     double lse = m + log(sum);
     for (int64_t j = 0; j < Sk; ++j)
-        p[j] = visible(i, j, Sq, Sk, causal) ? exp(s[j] - lse) : 0.0;
+        p[j] = visible(i, j, mk) ? exp(s[j] - lse) : 0.0;
     return lse;
 }
 
-static int check_args(const void *q, const void *k, const void *v, int64_t n_heads, int64_t Sq, int64_t Sk,
-                      int64_t D, const int64_t *rows, int64_t n_rows)
+static int check_args(const void *q, const void *k, const void *v, int64_t n_heads, int64_t n_kv_heads, int64_t Sq,
+                      int64_t Sk, int64_t D, const int64_t *rows, int64_t n_rows)
 {
     if (!q || !k || !v || !rows) return -1;
-    if (n_heads < 1 || Sq < 1 || Sk < 1 || D < 1 || n_rows < 0) return -1;
+    if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || Sq < 1 || Sk < 1 || D < 1 || n_rows < 0) return -1;
     for (int64_t t = 0; t < n_heads * n_rows; ++t)
         if (rows[t] < 0 || rows[t] >= Sq) return -1;
     return 0;
 }
 
-int oracle_attn_fwd(const double *q, const double *k, const double *v, int64_t n_heads, int64_t Sq, int64_t Sk,
-                    int64_t D, int causal, double scale, const int64_t *rows, int64_t n_rows, double *out,
-                    double *lse)
+int oracle_attn_fwd(const double *q, const double *k, const double *v, int64_t n_heads, int64_t n_kv_heads,
+                    int64_t Sq, int64_t Sk, int64_t D, int causal, int64_t window_left, int64_t window_right,
+                    double scale, const int64_t *rows, int64_t n_rows, double *out, double *lse)
 {
-    if (check_args(q, k, v, n_heads, Sq, Sk, D, rows, n_rows) || !out || !lse) return -1;
+    if (check_args(q, k, v, n_heads, n_kv_heads, Sq, Sk, D, rows, n_rows) || !out || !lse) return -1;
+    const struct mask mk = {Sq, Sk, causal, window_left, window_right};
+    const int64_t group = n_heads / n_kv_heads;
     int64_t total = n_heads * n_rows;
 #pragma omp parallel
     {
@@ -97,10 +116,10 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v, int64_t n
         for (int64_t t = 0; t < total; ++t) {
             int64_t h = t / n_rows;
             int64_t i = rows[t];
-            const double *kh = k + h * Sk * D;
-            const double *vh = v + h * Sk * D;
+            const double *kh = k + (h / group) * Sk * D;
+            const double *vh = v + (h / group) * Sk * D;
             row_scores(q + (h * Sq + i) * D, kh, Sk, D, scale, s);
-            lse[t] = row_softmax(s, i, Sq, Sk, causal, p);
+            lse[t] = row_softmax(s, i, &mk, p);
             double *o = out + t * D;
             for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
             for (int64_t j = 0; j < Sk; ++j)
@@ -113,10 +132,15 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v, int64_t n
 }
 
 int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout, int64_t n_heads,
-                    int64_t Sq, int64_t Sk, int64_t D, int causal, double scale, const int64_t *rows,
-                    int64_t n_rows, double *dq, double *dk, double *dv)
+                    int64_t n_kv_heads, int64_t Sq, int64_t Sk, int64_t D, int causal, int64_t window_left,
+                    int64_t window_right, double scale, const int64_t *rows, int64_t n_rows, double *dq, double *dk,
+                    double *dv)
 {
-    if (check_args(q, k, v, n_heads, Sq, Sk, D, rows, n_rows) || !dout || !dq || !dk || !dv) return -1;
+    if (check_args(q, k, v, n_heads, n_kv_heads, Sq, Sk, D, rows, n_rows) || !dout || !dq || !dk || !dv) return -1;
+    const struct mask mk = {Sq, Sk, causal, window_left, window_right};
+    const int64_t group = n_heads / n_kv_heads;
+    memset(dk, 0, sizeof(double) * (size_t)(n_kv_heads * Sk * D));
+    memset(dv, 0, sizeof(double) * (size_t)(n_kv_heads * Sk * D));
     /* Per head: P and dS of the listed rows, kept whole so that dK and dV are plain sums over rows. */
     double *P = (double *)malloc(sizeof(double) * (size_t)(n_rows ? n_rows : 1) * (size_t)Sk);
     double *dS = (double *)malloc(sizeof(double) * (size_t)(n_rows ? n_rows : 1) * (size_t)Sk);
@@ -127,8 +151,8 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
     }
     for (int64_t h = 0; h < n_heads; ++h) {
         const double *qh = q + h * Sq * D;
-        const double *kh = k + h * Sk * D;
-        const double *vh = v + h * Sk * D;
+        const double *kh = k + (h / group) * Sk * D;
+        const double *vh = v + (h / group) * Sk * D;
         const double *doh = dout + h * Sq * D;
         const int64_t *rh = rows + h * n_rows;
 #pragma omp parallel
@@ -141,7 +165,7 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
                 double *Pi = P + r * Sk;
                 double *dSi = dS + r * Sk;
                 row_scores(qh + i * D, kh, Sk, D, scale, s);
-                row_softmax(s, i, Sq, Sk, causal, Pi);
+                row_softmax(s, i, &mk, Pi);
                 /* dP_ij = dO_i . v_j */
                 for (int64_t j = 0; j < Sk; ++j) {
                     double acc = 0.0;
@@ -163,8 +187,9 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
             free(s);
             free(dP);
         }
-        double *dkh = dk + h * Sk * D;
-        double *dvh = dv + h * Sk * D;
+        /* this q head's contributions are added to its K/V head (a group shares one K/V head) */
+        double *dkh = dk + (h / group) * Sk * D;
+        double *dvh = dv + (h / group) * Sk * D;
 #pragma omp parallel for schedule(static)
         for (int64_t j = 0; j < Sk; ++j) {
             for (int64_t d = 0; d < D; ++d) {
@@ -175,8 +200,8 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
                     gk += dS[r * Sk + j] * qh[i * D + d];
                     gv += P[r * Sk + j] * doh[i * D + d];
                 }
-                dkh[j * D + d] = scale * gk;
-                dvh[j * D + d] = gv;
+                dkh[j * D + d] += scale * gk;
+                dvh[j * D + d] += gv;
             }
         }
     }

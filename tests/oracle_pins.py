@@ -16,7 +16,11 @@ What pins it:
   * a library routine the definition reduces to: torch's scaled_dot_product_attention on the CPU in
     float64, with autograd for the gradients (the skill page names SDPA in its quick start);
   * the causal reading for Sq != Sk (bottom-right aligned) and fully masked rows (O = 0, LSE = -inf);
-  * the default scale 1/sqrt(d): the skill page divides by 8.0 for d = 64 (Workflow 1, Step 3 and 4).
+  * the default scale 1/sqrt(d): the skill page divides by 8.0 for d = 64 (Workflow 1, Step 3 and 4);
+  * grouped K/V heads (skill page, Workflow 2 Step 3): the same as repeating each K/V head over its group
+    (dK/dV summed over the group), finite differences through the shared heads, and torch SDPA with
+    enable_gqa; the sliding window (Workflow 2 Steps 2-3, window_size=(left, right)): a window wider than the
+    sequence changes nothing, (0, 0) keeps only the aligned key, finite differences, SDPA with a band mask.
 """
 import json
 import math
@@ -253,8 +257,9 @@ def pin_golden_hand_examples(orc):
         cases = json.load(f)["cases"]
     for c in cases:
         q, k, v, do = (np.array(_parse(c[n]))[None] for n in ("q", "k", "v", "dout"))
-        out, lse = orc.fwd(q, k, v, causal=c["causal"], scale=c["scale"])
-        dq, dk, dv = orc.bwd(q, k, v, do, causal=c["causal"], scale=c["scale"])
+        win = tuple(c.get("window", (-1, -1)))
+        out, lse = orc.fwd(q, k, v, causal=c["causal"], scale=c["scale"], window=win)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=c["causal"], scale=c["scale"], window=win)
         _close(out[0], _parse(c["out"]), tol=1e-14, what=c["name"] + " O")
         _close(lse[0], _parse(c["lse"]), tol=1e-14, what=c["name"] + " LSE")
         _close(dq[0], _parse(c["dq"]), tol=1e-14, what=c["name"] + " dQ")
@@ -262,6 +267,127 @@ def pin_golden_hand_examples(orc):
         _close(dv[0], _parse(c["dv"]), tol=1e-14, what=c["name"] + " dV")
 
 
+def _repeat_heads(x, group):
+    return np.repeat(x, group, axis=0)
+
+
+def pin_gqa_matches_repeated_kv(orc):
+    r = _rng(12)
+    for causal, window in ((False, (-1, -1)), (True, (-1, -1)), (True, (2, 0)), (False, (1, 2))):
+        nq, nkv, Sq, Sk, D = 6, 2, 7, 9, 4
+        q = r.standard_normal((nq, Sq, D))
+        k = r.standard_normal((nkv, Sk, D))
+        v = r.standard_normal((nkv, Sk, D))
+        do = r.standard_normal((nq, Sq, D))
+        g = nq // nkv
+        o1, l1 = orc.fwd(q, k, v, causal=causal, scale=0.6, window=window)
+        o2, l2 = orc.fwd(q, _repeat_heads(k, g), _repeat_heads(v, g), causal=causal, scale=0.6, window=window)
+        _close(o1, o2, what="GQA O")
+        _close(l1, l2, what="GQA LSE")
+        dq1, dk1, dv1 = orc.bwd(q, k, v, do, causal=causal, scale=0.6, window=window)
+        dq2, dk2, dv2 = orc.bwd(q, _repeat_heads(k, g), _repeat_heads(v, g), do, causal=causal, scale=0.6,
+                                window=window)
+        _close(dq1, dq2, what="GQA dQ")
+        _close(dk1, dk2.reshape(nkv, g, Sk, D).sum(axis=1), what="GQA dK = group sum")
+        _close(dv1, dv2.reshape(nkv, g, Sk, D).sum(axis=1), what="GQA dV = group sum")
+
+
+def _fd_check(orc, q, k, v, do, causal, scale, window, what):
+    h = 1e-6
+    dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=scale, window=window)
+
+    def loss(qq, kk, vv):
+        out, _ = orc.fwd(qq, kk, vv, causal=causal, scale=scale, window=window)
+        return float(np.sum(out * do))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q, "k": k, "v": v}
+            xp = x.copy()
+            xp[idx] += h
+            xm = x.copy()
+            xm[idx] -= h
+            ap = dict(args, **{name: xp})
+            am = dict(args, **{name: xm})
+            num[idx] = (loss(ap["q"], ap["k"], ap["v"]) - loss(am["q"], am["k"], am["v"])) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        zero_ok = np.linalg.norm(num) < 1e-9 and np.linalg.norm(g) < 1e-9
+        assert zero_ok or err <= 1e-6, (what, "d" + name, err)
+
+
+def pin_gqa_and_window_finite_differences(orc):
+    r = _rng(13)
+    cases = [(4, 2, 4, 4, 2, False, (-1, -1)), (3, 1, 5, 5, 2, True, (-1, -1)), (2, 2, 6, 6, 2, True, (1, 0)),
+             (2, 1, 4, 6, 2, False, (1, 1)), (4, 2, 6, 4, 2, True, (2, -1))]
+    for (nq, nkv, Sq, Sk, D, causal, window) in cases:
+        q = r.standard_normal((nq, Sq, D))
+        k = r.standard_normal((nkv, Sk, D))
+        v = r.standard_normal((nkv, Sk, D))
+        do = r.standard_normal((nq, Sq, D))
+        _fd_check(orc, q, k, v, do, causal, 0.7, window, (nq, nkv, Sq, Sk, causal, window))
+
+
+def pin_window_limits(orc):
+    r = _rng(14)
+    q = r.standard_normal((2, 6, 3))
+    k = r.standard_normal((2, 8, 3))
+    v = r.standard_normal((2, 8, 3))
+    for causal in (False, True):
+        o1, l1 = orc.fwd(q, k, v, causal=causal, scale=0.5)
+        o2, l2 = orc.fwd(q, k, v, causal=causal, scale=0.5, window=(100, 100))
+        _close(o1, o2, what="wide window = no window")
+        _close(l1, l2, what="wide window LSE")
+    # (0, 0): only the aligned key c = i + Sk - Sq is visible
+    o, l = orc.fwd(q, k, v, causal=False, scale=0.5, window=(0, 0))
+    for i in range(6):
+        c = i + 2
+        _close(o[:, i], v[:, c], what="window (0,0) picks the aligned key")
+        _close(l[:, i], 0.5 * np.einsum("hd,hd->h", q[:, i], k[:, c]), what="window (0,0) LSE")
+    # rows whose window lies entirely outside the keys see nothing
+    o, l = orc.fwd(q[:, :1], k[:, :3], v[:, :3], causal=False, scale=0.5, window=(0, 0))  # c = 0 + 3 - 1 = 2
+    _close(o[:, 0], v[:, 2], what="window at the last key")
+    qq = r.standard_normal((1, 4, 3))
+    o, l = orc.fwd(qq, k[:1, :2], v[:1, :2], causal=True, scale=0.5, window=(0, 0))  # c = i - 2
+    assert np.all(o[0, :2] == 0) and np.all(np.isneginf(l[0, :2])), "window before the first key sees nothing"
+
+
+def pin_window_gqa_sdpa_crosscheck(orc):
+    import torch
+
+    r = _rng(15)
+    for (nq, nkv, Sq, Sk, D, causal, window) in ((4, 2, 12, 12, 8, True, (3, 0)), (4, 4, 10, 14, 4, False, (2, 3)),
+                                                  (6, 3, 9, 9, 4, True, (-1, -1)), (2, 1, 7, 5, 4, False, (1, -1))):
+        q = r.standard_normal((nq, Sq, D))
+        k = r.standard_normal((nkv, Sk, D))
+        v = r.standard_normal((nkv, Sk, D))
+        do = r.standard_normal((nq, Sq, D))
+        i = torch.arange(Sq)[:, None]
+        j = torch.arange(Sk)[None, :]
+        c = i + (Sk - Sq)
+        mask = torch.ones(Sq, Sk, dtype=torch.bool)
+        if causal:
+            mask &= j <= c
+        if window[0] >= 0:
+            mask &= j >= c - window[0]
+        if window[1] >= 0:
+            mask &= j <= c + window[1]
+        tq = torch.tensor(q[None], requires_grad=True)
+        tk = torch.tensor(k[None], requires_grad=True)
+        tv = torch.tensor(v[None], requires_grad=True)
+        o_ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, enable_gqa=True)
+        o_ref.backward(torch.tensor(do[None]))
+        rows_ok = mask.any(dim=1).numpy()
+        out, _ = orc.fwd(q, k, v, causal=causal, window=window)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, window=window)
+        _close(out[:, rows_ok], o_ref.detach()[0].numpy()[:, rows_ok], what="SDPA GQA/window O")
+        if rows_ok.all():
+            _close(dq, tq.grad[0].numpy(), what="SDPA GQA/window dQ")
+            _close(dk, tk.grad[0].numpy(), what="SDPA GQA/window dK")
+            _close(dv, tv.grad[0].numpy(), what="SDPA GQA/window dV")
+
+
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
-            pin_causal_alignment, pin_default_scale, pin_golden_hand_examples]
+            pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
+            pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck]

@@ -15,8 +15,14 @@ SRC = os.path.join(ROOT, "oracle", "fa_oracle.c")
 
 MUTANTS = {
     "drop_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
-    "causal_off_by_one": ("return j <= i + (Sk - Sq);", "return j < i + (Sk - Sq);"),
-    "causal_top_left": ("return j <= i + (Sk - Sq);", "return j <= i;"),
+    "causal_off_by_one": ("if (m->causal && j > c) return 0;", "if (m->causal && j >= c) return 0;"),
+    "causal_top_left": ("int64_t c = i + (m->Sk - m->Sq);", "int64_t c = i;"),
+    "window_left_off_by_one": ("if (m->left >= 0 && j < c - m->left) return 0;",
+                               "if (m->left >= 0 && j <= c - m->left) return 0;"),
+    "window_right_ignored": ("if (m->right >= 0 && j > c + m->right) return 0;", ""),
+    "gqa_wrong_kv_head": ("const double *kh = k + (h / group) * Sk * D;\n            const double *vh = v + (h / group) * Sk * D;",
+                          "const double *kh = k + (h % n_kv_heads) * Sk * D;\n            const double *vh = v + (h % n_kv_heads) * Sk * D;"),
+    "gqa_dk_not_summed": ("dkh[j * D + d] += scale * gk;", "dkh[j * D + d] = scale * gk;"),
     "lse_drops_max": ("double lse = m + log(sum);", "double lse = log(sum);"),
     "output_uses_k": ("o[d] += p[j] * vh[j * D + d];", "o[d] += p[j] * kh[j * D + d];"),
     "dp_uses_k": ("acc += doh[i * D + d] * vh[j * D + d];", "acc += doh[i * D + d] * kh[j * D + d];"),
@@ -26,7 +32,7 @@ MUTANTS = {
     "dq_uses_v": ("dqi[d] += dSi[j] * kh[j * D + d];", "dqi[d] += dSi[j] * vh[j * D + d];"),
     "dk_uses_dout": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * doh[i * D + d];"),
     "dv_uses_dS": ("gv += P[r * Sk + j] * doh[i * D + d];", "gv += dS[r * Sk + j] * doh[i * D + d];"),
-    "dk_no_scale": ("dkh[j * D + d] = scale * gk;", "dkh[j * D + d] = gk;"),
+    "dk_no_scale": ("dkh[j * D + d] += scale * gk;", "dkh[j * D + d] += gk;"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
