@@ -4,11 +4,13 @@ Every step of the computation runs in the library's CUDA kernels; this module on
 (PyTorch tensors -> device pointers, sizes and the current CUDA stream) and turns status codes into
 exceptions. There is no fallback: if the library is missing or fails to load, every call raises.
 
-    fwd(q, k, v, causal=False, scale=None) -> (out, lse)
-    bwd(q, k, v, out, lse, dout, causal=False, scale=None) -> (dq, dk, dv)
+    fwd(q, k, v, causal=False, scale=None, window=(-1, -1)) -> (out, lse)
+    bwd(q, k, v, out, lse, dout, causal=False, scale=None, window=(-1, -1)) -> (dq, dk, dv)
 
-Layouts follow the C header (include/fa.h): q/out/dout [B, Sq, H, D], k/v [B, Sk, H, D], fp16 or bf16,
-contiguous, on one CUDA device; lse is fp32 [B, H, Sq]. ``scale=None`` means 1/sqrt(D).
+Layouts follow the C header (include/fa.h): q/out/dout [B, Sq, H, D], k/v [B, Sk, Hkv, D] (Hkv divides H:
+grouped or multi-query K/V heads), fp16 or bf16, contiguous, on one CUDA device; lse is fp32 [B, H, Sq].
+``scale=None`` means 1/sqrt(D); ``window=(left, right)`` limits each query to keys within left before and
+right after its aligned key (-1 = unbounded side).
 """
 import ctypes
 import os
@@ -20,7 +22,8 @@ FA_F16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
                 -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
-EXPORTS = ("fa_fwd", "fa_bwd", "fa_bwd_stage", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status")
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
+           "fa_status_string", "fa_device_status")
 
 _lib = None
 
@@ -47,6 +50,10 @@ def lib():
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_bwd_stage.restype = i
     L.fa_bwd_stage.argtypes = [i] + L.fa_bwd.argtypes
+    L.fa_fwd_ex.restype = i
+    L.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp]
+    L.fa_bwd_ex.restype = i
+    L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_status_string.restype = ctypes.c_char_p
@@ -85,7 +92,7 @@ def _check_bshd(name, t, dev):
         raise ValueError("%s must be a contiguous [B, S, H, D] tensor" % name)
 
 
-def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, window=(-1, -1)):
     """Forward attention. Returns (out [B,Sq,H,D] in q's dtype, lse fp32 [B,H,Sq])."""
     import torch
 
@@ -98,10 +105,12 @@ def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
-    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, D,
-                      int(bool(causal)), float(0.0 if scale is None else scale), _dtype_code(q), _stream_ptr(stream))
+    Hkv = k.shape[2]
+    rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, Hkv,
+                         D, int(bool(causal)), int(window[0]), int(window[1]), float(0.0 if scale is None else scale),
+                         _dtype_code(q), _stream_ptr(stream))
     if rc != FA_OK:
-        raise FAError(rc, "fa_fwd")
+        raise FAError(rc, "fa_fwd_ex")
     return out, lse
 
 
@@ -110,7 +119,7 @@ def workspace_size(B, Sq, H, D):
 
 
 def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None,
-        stage=-1):
+        stage=-1, window=(-1, -1)):
     """Backward attention (P recomputed from lse). Returns (dq, dk, dv) in q's dtype.
 
     ``stage`` selects one of the three launches (0 preprocess, 1 main, 2 dQ conversion; -1 all), see
@@ -128,10 +137,19 @@ def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=
     ws_bytes = workspace_size(B, Sq, H, D)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = lib().fa_bwd_stage(int(stage), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D,
-                            int(bool(causal)), float(0.0 if scale is None else scale), _dtype_code(q),
-                            workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    Hkv = k.shape[2]
+    sc = float(0.0 if scale is None else scale)
+    ws_args = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if stage == -1:
+        rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, Hkv, D, int(bool(causal)),
+                             int(window[0]), int(window[1]), sc, _dtype_code(q), *ws_args)
+    else:
+        if Hkv != H or tuple(window) != (-1, -1):
+            raise ValueError("single backward stages are available for plain attention only")
+        rc = lib().fa_bwd_stage(int(stage), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D,
+                                int(bool(causal)), sc, _dtype_code(q), *ws_args)
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
     return dq, dk, dv

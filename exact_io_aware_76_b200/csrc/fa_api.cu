@@ -156,7 +156,7 @@ int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
-    kern<<<(unsigned)(p.n_kblk * p.B * p.H), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<(unsigned)(p.n_kblk * p.B * p.Hkv), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {
@@ -201,10 +201,12 @@ int fa_device_status(int reset) {
   return v;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H, int D,
-           int causal, float scale, int dtype, cudaStream_t stream) {
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
+              int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+              cudaStream_t stream) {
   if (!q || !k || !v || !out || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return FA_ERR_INVALID;
+  if (Hkv < 1 || H < 1 || H % Hkv != 0) return FA_ERR_INVALID;
   int rc = check_common(B, Sq, Sk, H, D, scale, dtype);
   if (rc) return rc;
   int dev = 0;
@@ -213,19 +215,23 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
 
   CUtensorMap tq, tk, tv;
   if ((rc = make_bshd_map(&tq, q, B, Sq, H, D, dtype, 128))) return rc;
-  if ((rc = make_bshd_map(&tk, k, B, Sk, H, D, dtype, 128))) return rc;
-  if ((rc = make_bshd_map(&tv, v, B, Sk, H, D, dtype, 128))) return rc;
+  if ((rc = make_bshd_map(&tk, k, B, Sk, Hkv, D, dtype, 128))) return rc;
+  if ((rc = make_bshd_map(&tv, v, B, Sk, Hkv, D, dtype, 128))) return rc;
   FwdParams p;
   p.out = out;
   p.lse = lse;
   p.B = B;
   p.H = H;
+  p.Hkv = Hkv;
+  p.group = H / Hkv;
+  p.win_left = window_left < 0 ? -1 : window_left;
+  p.win_right = window_right < 0 ? -1 : window_right;
   p.Sq = Sq;
   p.Sk = Sk;
   p.n_qblk = (Sq + 255) / 256;
   p.n_kv_total = (Sk + 127) / 128;
   // Head-major CTA order once a head's re-read K/V no longer fit in L2 together with the other heads'.
-  p.head_major = (2.0 * B * Sk * H * D * 2 > kHeadMajorBytes) ? 1 : 0;
+  p.head_major = (2.0 * B * Sk * Hkv * D * 2 > kHeadMajorBytes) ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
   const bool c = causal != 0;
   if (D == 64)
@@ -235,15 +241,22 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
                           : dispatch_fwd_causal<128, false>(c, tq, tk, tv, p, dev, stream);
 }
 
+int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H, int D,
+           int causal, float scale, int dtype, cudaStream_t stream) {
+  return fa_fwd_ex(q, k, v, out, lse, B, Sq, Sk, H, H, D, causal, -1, -1, scale, dtype, stream);
+}
+
 size_t fa_bwd_workspace_size(int B, int Sq, int H, int D) {
   if (check_common(B, Sq, 1, H, D, 1.f, FA_F16) != FA_OK) return 0;
   return bwd_layout(B, Sq, H, D).total;
 }
 
-int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
-                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal,
-                 float scale, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+static int bwd_impl(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D,
+                    int causal, int window_left, int window_right, float scale, int dtype, void* workspace,
+                    size_t workspace_bytes, cudaStream_t stream) {
   if (stage < -1 || stage > 2) return FA_ERR_INVALID;
+  if (Hkv < 1 || H < 1 || H % Hkv != 0) return FA_ERR_INVALID;
   const void* ptrs[9] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!ptr || !aligned16(ptr)) return FA_ERR_INVALID;
@@ -260,8 +273,8 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
   CUtensorMap tq, tk, tv, tdo;
   if ((rc = make_bshd_map(&tq, q, B, Sq, H, D, dtype, bq))) return rc;
   if ((rc = make_bshd_map(&tdo, dout, B, Sq, H, D, dtype, bq))) return rc;
-  if ((rc = make_bshd_map(&tk, k, B, Sk, H, D, dtype, 128))) return rc;
-  if ((rc = make_bshd_map(&tv, v, B, Sk, H, D, dtype, 128))) return rc;
+  if ((rc = make_bshd_map(&tk, k, B, Sk, Hkv, D, dtype, 128))) return rc;
+  if ((rc = make_bshd_map(&tv, v, B, Sk, Hkv, D, dtype, 128))) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   BwdParams p;
   p.out = out;
@@ -275,6 +288,10 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
   p.lse2 = reinterpret_cast<float*>(ws + lay.lse2);
   p.B = B;
   p.H = H;
+  p.Hkv = Hkv;
+  p.group = H / Hkv;
+  p.win_left = window_left < 0 ? -1 : window_left;
+  p.win_right = window_right < 0 ? -1 : window_right;
   p.Sq = Sq;
   p.Sk = Sk;
   p.Sq_pad = lay.sq_pad;
@@ -289,6 +306,21 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
                             : dispatch_bwd_causal<64, false>(stage, c, tq, tk, tv, tdo, p, dev, stream);
   return dtype == FA_BF16 ? dispatch_bwd_causal<128, true>(stage, c, tq, tk, tv, tdo, p, dev, stream)
                           : dispatch_bwd_causal<128, false>(stage, c, tq, tk, tv, tdo, p, dev, stream);
+}
+
+int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal,
+                 float scale, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_impl(stage, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, H, D, causal, -1, -1, scale, dtype,
+                  workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+              void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D, int causal, int window_left,
+              int window_right, float scale, int dtype, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream) {
+  return bwd_impl(-1, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, Hkv, D, causal, window_left, window_right,
+                  scale, dtype, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout, void* dq,

@@ -38,13 +38,15 @@ struct BwdParams {
   const void* out;   // [B,Sq,H,D]
   const void* dout;  // [B,Sq,H,D]
   const float* lse;  // [B,H,Sq]
-  void* dk;          // [B,Sk,H,D]
-  void* dv;          // [B,Sk,H,D]
+  void* dk;          // [B,Sk,Hkv,D]
+  void* dv;          // [B,Sk,Hkv,D]
   void* dq;          // [B,Sq,H,D]
   float* dq_acc;     // [B,H,Sq_pad,D] fp32
   float* dvec;       // [B,H,Sq_pad]   D_i
   float* lse2;       // [B,H,Sq_pad]   LSE_i * log2(e), +inf for padding rows and rows without keys
-  int B, H, Sq, Sk, Sq_pad;
+  int B, H, Sq, Sk, Sq_pad;  // H = query heads
+  int Hkv, group;            // K/V heads and query heads per K/V head (H = Hkv * group)
+  int win_left, win_right;   // window around the aligned key i + Sk - Sq; negative = unbounded side
   int n_kblk;        // ceil(Sk / 128)
   int head_major;    // CTA order: 1 = all key tiles of a head together (L2 reuse), 0 = heavy-first
   float scale, scale_log2;
@@ -188,19 +190,25 @@ __global__ void __launch_bounds__(384, 1)
   // CTA order. Head-major (large problems): the key tiles of one (batch, head) run together, so its Q, dO and
   // fp32 dQ accumulator stay resident in L2 while every key tile reads them and reduces into them; heavy-first
   // within the head (the first key tiles are seen by the most query tiles). Otherwise heavy-first across heads.
-  const int n_bh = p.B * p.H;
-  const int bh = p.head_major ? blockIdx.x / p.n_kblk : blockIdx.x % n_bh;
+  // A CTA owns one (batch, K/V head, key tile) and walks every query head of the K/V head's group, so the
+  // group's dK/dV contributions accumulate in TMEM without any further reduction.
+  const int n_bh = p.B * p.Hkv;
+  const int bh = p.head_major ? blockIdx.x / p.n_kblk : blockIdx.x % n_bh;  // (batch, K/V head)
   const int kblk = p.head_major ? blockIdx.x % p.n_kblk : blockIdx.x / n_bh;
-  const int b = bh / p.H, h = bh % p.H;
+  const int b = bh / p.Hkv, h_kv = bh % p.Hkv;
   const int off = p.Sk - p.Sq;
   const int key0 = kblk * 128;
-  const int n_qtiles = (p.Sq + BQ - 1) / BQ;
-  int i_begin = 0;
-  if (kCausal) {
-    const int q_min = key0 - off;  // the first query that sees key0
-    i_begin = q_min <= 0 ? 0 : q_min / BQ;
-  }
-  const int n_it = max(0, n_qtiles - i_begin);
+  const int key1 = min(p.Sk - 1, key0 + 127);
+  // Query r sees key j iff r + off - left <= j <= r + off + right (causal caps right at 0; negative bounds are
+  // unbounded), i.e. j - off - right <= r <= j - off + left.
+  const bool has_left = p.win_left >= 0;
+  const int right = kCausal ? (p.win_right >= 0 ? min(p.win_right, 0) : 0) : p.win_right;
+  const bool has_right = right >= 0;
+  const int r_min = has_right ? max(0, key0 - off - right) : 0;
+  const int r_max = has_left ? min(p.Sq - 1, key1 - off + p.win_left) : p.Sq - 1;
+  const int i_begin = r_min / BQ;
+  const int n_q = (r_max >= r_min) ? r_max / BQ - i_begin + 1 : 0;  // query tiles per head
+  const int n_it = n_q * p.group;                                     // iteration it: head it / n_q
 
   const uint32_t warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -228,7 +236,6 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
-  const size_t bh_row0 = static_cast<size_t>(bh) * p.Sq_pad;
 
   if (warp >= 8) {
     regs_dec<L::kRegsOther>();
@@ -240,21 +247,23 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(kv_full, 2 * L::kKVBytes);
       for (int c = 0; c < L::kChunks; ++c) {
-        tma_load_4d(smem + L::kKOff + c * 16384, &tm_k, kv_full, 64 * c, h, key0, b);
-        tma_load_4d(smem + L::kVOff + c * 16384, &tm_v, kv_full, 64 * c, h, key0, b);
+        tma_load_4d(smem + L::kKOff + c * 16384, &tm_k, kv_full, 64 * c, h_kv, key0, b);
+        tma_load_4d(smem + L::kVOff + c * 16384, &tm_v, kv_full, 64 * c, h_kv, key0, b);
       }
       int it = 0;
       for (; it < n_it; ++it) {
         const int s = it % NQS;
-        const int q0 = (i_begin + it) * BQ;
+        const int h = h_kv * p.group + it / n_q;
+        const int q0 = (i_begin + it % n_q) * BQ;
+        const size_t row0 = (static_cast<size_t>(b) * p.H + h) * p.Sq_pad + q0;
         if (it >= NQS && !mbar_wait(&q_empty[s], ((it / NQS) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[s], 2 * L::kQBytes + 2 * BQ * 4);
         for (int c = 0; c < L::kChunks; ++c) {
           tma_load_4d(smem + L::kQOff + s * L::kQBytes + c * BQ * 128, &tm_q, &q_full[s], 64 * c, h, q0, b);
           tma_load_4d(smem + L::kDOOff + s * L::kQBytes + c * BQ * 128, &tm_do, &q_full[s], 64 * c, h, q0, b);
         }
-        bulk_load(smem + L::kLOff + s * BQ * 4, p.lse2 + bh_row0 + q0, BQ * 4, &q_full[s]);
-        bulk_load(smem + L::kDVecOff + s * BQ * 4, p.dvec + bh_row0 + q0, BQ * 4, &q_full[s]);
+        bulk_load(smem + L::kLOff + s * BQ * 4, p.lse2 + row0, BQ * 4, &q_full[s]);
+        bulk_load(smem + L::kDVecOff + s * BQ * 4, p.dvec + row0, BQ * 4, &q_full[s]);
       }
       if (*abort_flag) {
         int drain = 0;
@@ -353,9 +362,11 @@ __global__ void __launch_bounds__(384, 1)
     const int key = key0 + j;
     const uint32_t lane_base = tmem + ((warp * 32) << 16);
     bool ok = true;
+    // Visible queries of this key: [key - off - right, key - off + left]; columns of a tile starting at q0
+    // are masked outside [lo_c, hi_c].
     for (int it = 0; it < n_it; ++it) {
       const int x = it % NB, s = it % NQS;
-      const int q0 = (i_begin + it) * BQ;
+      const int q0 = (i_begin + it % n_q) * BQ;
       if (!mbar_wait(&sdp_full[x], (it / NB) & 1, abort_flag)) { ok = false; break; }
       if (it >= NB && !mbar_wait(&ds_empty[x], ((it / NB) - 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after_sync();
@@ -363,9 +374,10 @@ __global__ void __launch_bounds__(384, 1)
       const float* dvec = reinterpret_cast<const float*>(smem + L::kDVecOff + s * BQ * 4);
       uint8_t* ds_row_base = smem + L::kDSOff + x * L::kDSBytes + j * 128;
       const uint32_t s_col = L::kColS + x * BQ, dp_col = L::kColDP + x * BQ;
-      // Keys visible to query q satisfy key <= q + off, i.e. column c >= lo.
-      const int lo = kCausal ? (key - off - q0) : -1;
-      const bool need_mask = kCausal && (key0 + 127 > q0 + off);
+      const int lo_c = has_right ? key - off - right - q0 : -1;
+      const int hi_c = has_left ? key - off + p.win_left - q0 : BQ;
+      // Whole tile visible to every key of this CTA: no element mask.
+      const bool need_mask = (has_right && key0 + 127 - off - right > q0) || (has_left && key0 - off + p.win_left < q0 + BQ - 1);
 #pragma unroll
       for (int c0 = 0; c0 < BQ; c0 += 64) {
         float sv[64], dp[64];
@@ -381,10 +393,10 @@ __global__ void __launch_bounds__(384, 1)
           float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l4.z));
           float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l4.w));
           if (need_mask) {
-            if (c0 + c < lo) p0 = 0.f;
-            if (c0 + c + 1 < lo) p1 = 0.f;
-            if (c0 + c + 2 < lo) p2 = 0.f;
-            if (c0 + c + 3 < lo) p3 = 0.f;
+            if (c0 + c < lo_c || c0 + c > hi_c) p0 = 0.f;
+            if (c0 + c + 1 < lo_c || c0 + c + 1 > hi_c) p1 = 0.f;
+            if (c0 + c + 2 < lo_c || c0 + c + 2 > hi_c) p2 = 0.f;
+            if (c0 + c + 3 < lo_c || c0 + c + 3 > hi_c) p3 = 0.f;
           }
           pk[c / 2] = pack2<kBF16>(p0, p1);
           pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
@@ -414,7 +426,7 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after_sync();
       const bool valid = key < p.Sk;
-      const size_t row_off = ((static_cast<size_t>(b) * p.Sk + key) * p.H + h) * D;
+      const size_t row_off = ((static_cast<size_t>(b) * p.Sk + key) * p.Hkv + h_kv) * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         uint16_t* dst = reinterpret_cast<uint16_t*>(which == 0 ? p.dv : p.dk) + row_off;
@@ -451,7 +463,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = tmem + ((quarter * 32) << 16);
     for (int it = 0; it < n_it; ++it) {
       const int x = it % NB;
-      const int q0 = (i_begin + it) * BQ;
+      const int h = h_kv * p.group + it / n_q;
+      const int q0 = (i_begin + it % n_q) * BQ;
+      const size_t row0 = (static_cast<size_t>(b) * p.H + h) * p.Sq_pad + q0;
       if (!mbar_wait(&dq_full[x], (it / NB) & 1, abort_flag)) break;
       tc_fence_after_sync();
       float v[64];
@@ -461,12 +475,12 @@ __global__ void __launch_bounds__(384, 1)
       if (D == 128) {
         // lane r = head-dim index, column = query: for each query the 32 lanes of a warp add to 128 contiguous
         // bytes (one coalesced reduction per query).
-        float* base = p.dq_acc + (bh_row0 + q0) * D + r;
+        float* base = p.dq_acc + row0 * D + r;
 #pragma unroll
         for (int c = 0; c < 64; ++c) atomicAdd(base + static_cast<size_t>(c) * D, v[c]);
       } else {
         // lane r = query row, column = head-dim index: 16-byte vector reductions along the row.
-        float* base = p.dq_acc + (bh_row0 + q0 + r) * D;
+        float* base = p.dq_acc + (row0 + r) * D;
 #pragma unroll
         for (int c = 0; c < 64; c += 4) red_add_v4(base + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
       }

@@ -38,7 +38,9 @@ constexpr float kRescaleLog2 = 8.0f;
 struct FwdParams {
   void* out;
   float* lse;
-  int B, H, Sq, Sk;
+  int B, H, Sq, Sk;    // H = query heads
+  int Hkv, group;      // K/V heads and query heads per K/V head (H = Hkv * group)
+  int win_left, win_right;  // window around the aligned key i + Sk - Sq; negative = unbounded side
   int n_qblk;      // ceil(Sq / 256)
   int n_kv_total;  // ceil(Sk / 128)
   int head_major;  // CTA order: 1 = all query blocks of a head together (K/V reuse in L2), 0 = heavy-first
@@ -92,24 +94,43 @@ __global__ void __launch_bounds__(384, 1)
   const int qblk_rank = p.head_major ? blockIdx.x % p.n_qblk : blockIdx.x / n_bh;
   const int qblk = kCausal ? (p.n_qblk - 1 - qblk_rank) : qblk_rank;
   const int b = bh / p.H, h = bh % p.H;
-  const int off = p.Sk - p.Sq;  // bottom-right alignment of the causal mask
+  const int h_kv = h / p.group;  // grouped heads: this q head reads K/V head h / group
+  const int off = p.Sk - p.Sq;   // bottom-right alignment of the causal mask and the window
+  // Visible keys of query row r: [r + off - left, r + off + right] within [0, Sk); the causal mask caps right
+  // at 0; a negative bound (and right without the causal mask) is unbounded.
+  const bool has_left = p.win_left >= 0;
+  const int right = kCausal ? (p.win_right >= 0 ? min(p.win_right, 0) : 0) : p.win_right;
+  const bool has_right = right >= 0;
 
-  // Number of key tiles each Q tile visits (0: tile beyond Sq, or no visible key at all).
-  int n_kv[2];
+  // Key tiles [j_lo[t], j_lo[t] + n_kv[t]) each Q tile visits (n_kv = 0: tile beyond Sq or no visible key).
+  int j_lo[2], n_kv[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int row0 = qblk * 256 + t * 128;
-    if (row0 >= p.Sq) {
+    const int row1 = min(p.Sq - 1, row0 + 127);
+    const int key_lo = has_left ? max(0, row0 + off - p.win_left) : 0;
+    const int key_hi = has_right ? min(p.Sk - 1, row1 + off + right) : p.Sk - 1;
+    if (row0 >= p.Sq || key_hi < key_lo) {
+      j_lo[t] = 0;
       n_kv[t] = 0;
-    } else if (kCausal) {
-      const int last_row = min(p.Sq - 1, row0 + 127);
-      const int last_key = last_row + off;
-      n_kv[t] = last_key < 0 ? 0 : min(p.n_kv_total, last_key / 128 + 1);
     } else {
-      n_kv[t] = p.n_kv_total;
+      j_lo[t] = key_lo / 128;
+      n_kv[t] = key_hi / 128 - j_lo[t] + 1;
     }
   }
-  const int n_iter = max(n_kv[0], n_kv[1]);
+  // The CTA walks the union of both intervals (contiguous: tile 1's rows follow tile 0's).
+  int j_begin, j_end;
+  if (n_kv[0] == 0) {
+    j_begin = j_lo[1];
+    j_end = j_lo[1] + n_kv[1];
+  } else if (n_kv[1] == 0) {
+    j_begin = j_lo[0];
+    j_end = j_lo[0] + n_kv[0];
+  } else {
+    j_begin = min(j_lo[0], j_lo[1]);
+    j_end = max(j_lo[0] + n_kv[0], j_lo[1] + n_kv[1]);
+  }
+  const int n_iter = j_end - j_begin;
 
   const uint32_t warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -155,16 +176,17 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(smem + L::kQOff + t * L::kTileBytes + c * 16384, &tm_q, q_full, 64 * c, h,
                       qblk * 256 + t * 128, b);
       }
-      int j = 0;
+      int j = 0;  // index into the CTA's key tiles; the key tile is j_begin + j
       for (; j < n_iter; ++j) {
         const int s = j % L::kStages;
+        const int key0 = (j_begin + j) * 128;
         if (j >= L::kStages && !mbar_wait(&kv_empty[s], ((j / L::kStages) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kKOff + s * L::kTileBytes + c * 16384, &tm_k, &k_full[s], 64 * c, h, j * 128, b);
+          tma_load_4d(smem + L::kKOff + s * L::kTileBytes + c * 16384, &tm_k, &k_full[s], 64 * c, h_kv, key0, b);
         mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kVOff + s * L::kTileBytes + c * 16384, &tm_v, &v_full[s], 64 * c, h, j * 128, b);
+          tma_load_4d(smem + L::kVOff + s * L::kTileBytes + c * 16384, &tm_v, &v_full[s], 64 * c, h_kv, key0, b);
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA exits (bounded; own flag, not the CTA's).
@@ -210,28 +232,30 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < 128 / 16; ++kk)
           umma_ts(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * 2048), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag);
-      if (ok) {
-        tc_fence_after_sync();
-        for (int t = 0; t < 2; ++t)
-          if (n_kv[t] > 0) {
-            issue_qk(t, 0);
-            umma_commit(&s_full[t]);
-          }
-      }
+      // Key tile jj (local index j = jj - j_begin) serves Q tile t when j_lo[t] <= jj < j_lo[t] + n_kv[t]; a
+      // tile's first S is issued when the walk reaches its interval, every later one right after its PV.
       for (int j = 0; ok && j < n_iter; ++j) {
+        const int jj = j_begin + j;
         const int s = j % L::kStages;
         const uint32_t ph = (j / L::kStages) & 1;
+        if (!mbar_wait(&k_full[s], ph, abort_flag)) break;
+        tc_fence_after_sync();
+        for (int t = 0; t < 2; ++t)
+          if (n_kv[t] > 0 && jj == j_lo[t]) {
+            issue_qk(t, s);
+            umma_commit(&s_full[t]);
+          }
         if (!mbar_wait(&v_full[s], ph, abort_flag)) break;
         const int jn = j + 1;
         bool next_k_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_kv[t]) continue;
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag)) { ok = false; break; }
+          if (n_kv[t] == 0 || jj < j_lo[t] || jj >= j_lo[t] + n_kv[t]) continue;
+          const int u = jj - j_lo[t];  // this tile's local step
+          if (!mbar_wait(&p_full[t], u & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_pv(t, s, j > 0);
+          issue_pv(t, s, u > 0);
           umma_commit(&o_full[t]);
-          if (jn < n_kv[t]) {
+          if (u + 1 < n_kv[t]) {
             if (!next_k_ready) {
               if (!mbar_wait(&k_full[jn % L::kStages], (jn / L::kStages) & 1, abort_flag)) { ok = false; break; }
               tc_fence_after_sync();
@@ -262,6 +286,13 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_tmem = lane_base + 256 + t * D;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // This row's visible keys (the causal mask and the window, clipped to [0, Sk)).
+    const int row_lo = has_left ? row + off - p.win_left : 0;
+    const int row_hi = has_right ? min(p.Sk - 1, row + off + right) : p.Sk - 1;
+    // Key tiles that lie wholly inside every row's range need no element mask.
+    const int tile_row0 = qblk * 256 + t * 128;
+    const int all_lo = has_left ? tile_row0 + 127 + off - p.win_left : 0;
+    const int all_hi = has_right ? min(p.Sk - 1, tile_row0 + off + right) : p.Sk - 1;
     for (int j = 0; j < nt; ++j) {
       if (!mbar_wait(&s_full[t], j & 1, abort_flag)) { ok = false; break; }
       // PV(j-1) completed before S(j) (in-order tensor pipe); waiting keeps the o_full phases in step.
@@ -269,13 +300,12 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after_sync();
       float s[128];
       tmem_ld_x128(s_tmem, reinterpret_cast<uint32_t*>(s));
-      const int key0 = j * 128;
-      const bool need_mask = (key0 + 128 > p.Sk) || (kCausal && key0 + 127 > qblk * 256 + t * 128 + off);
+      const int key0 = (j_lo[t] + j) * 128;
+      const bool need_mask = key0 < all_lo || key0 + 127 > all_hi;
       if (need_mask) {
-        const int lim = kCausal ? min(p.Sk - 1, row + off) : (p.Sk - 1);  // last visible key of this row
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (key0 + c > lim) s[c] = -INFINITY;
+          if (key0 + c < row_lo || key0 + c > row_hi) s[c] = -INFINITY;
       }
       float mx = s[0];
 #pragma unroll
@@ -284,7 +314,9 @@ __global__ void __launch_bounds__(384, 1)
       // Warp-uniform decision: TMEM loads/stores below are warp-collective.
       const bool rescale = __any_sync(0xffffffffu, m_cand > m + kRescaleLog2);
       if (rescale) {
-        const float alpha = ex2_approx(m - m_cand);  // 0 when m == -inf
+        // A row that has not seen a visible key yet (m = -inf) has O = 0 and l = 0; the warp may rescale
+        // because of other rows, and 2^(m - m_cand) would be 2^(-inf + inf) = NaN for it when m_cand is -inf.
+        const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_cand);
         if (j > 0) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {

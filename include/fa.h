@@ -69,6 +69,21 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* out, float*
            int causal, float scale, int dtype, cudaStream_t stream);
 
 /*
+ * Forward with grouped K/V heads and a sliding window (skill page "Flash Attention — …", Workflow 2 Step 3:
+ * multi-query attention with fewer KV heads, and Steps 2-3: window_size=(left, right)).
+ *   H query heads, Hkv K/V heads (H a multiple of Hkv; Hkv = 1 is multi-query): query head h reads K/V head
+ *   h / (H / Hkv); k and v are [B, Sk, Hkv, D].
+ *   window_left, window_right: with c = i + Sk - Sq the key aligned with query i, key j is visible iff
+ *   (window_left < 0 or j >= c - window_left) and (window_right < 0 or j <= c + window_right), on top of the
+ *   causal rule (which caps the right side at c). Negative = unbounded ((-1, -1) = no window).
+ * fa_fwd(..., H, ...) is fa_fwd_ex(..., H, H, ..., -1, -1, ...). Other conventions as above; additionally
+ * FA_ERR_INVALID if Hkv < 1 or H is not a multiple of Hkv.
+ */
+FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                     int H, int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+                     cudaStream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes (0 on invalid sizes). The workspace holds the fp32
  * dQ accumulator and the per-row fp32 terms D_i = rowsum(dO_i * O_i) and LSE_i * log2(e).
  */
@@ -85,6 +100,16 @@ FA_API size_t fa_bwd_workspace_size(int B, int Sq, int H, int D);
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
            void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal, float scale, int dtype,
            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward with grouped K/V heads and a sliding window (same arguments and readings as fa_fwd_ex): dk and dv
+ * are [B, Sk, Hkv, D], each K/V head's gradient summed over its group of query heads; dq is [B, Sq, H, D].
+ * The workspace size is fa_bwd_workspace_size(B, Sq, H, D) with H the number of query heads.
+ */
+FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D,
+                     int causal, int window_left, int window_right, float scale, int dtype, void* workspace,
+                     size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * The three launches of fa_bwd one at a time, for callers that time or schedule them separately:

@@ -30,14 +30,31 @@ def all_heads(B, H):
     return [(b, h) for b in range(B) for h in range(H)]
 
 
-def oracle_fwd(q, k, v, causal, scale, heads, rows=None):
-    return oracle.attn_fwd(heads_f64(q, heads), heads_f64(k, heads), heads_f64(v, heads), causal=causal,
-                           scale=scale, rows=rows)
+def kv_heads(q, k, heads):
+    """The K/V head each query head of ``heads`` reads (grouped heads: h // (Hq / Hkv))."""
+    group = q.shape[2] // k.shape[2]
+    return [(b, h // group) for (b, h) in heads]
 
 
-def oracle_bwd(q, k, v, do, causal, scale, heads, rows=None):
-    return oracle.attn_bwd(heads_f64(q, heads), heads_f64(k, heads), heads_f64(v, heads), heads_f64(do, heads),
-                           causal=causal, scale=scale, rows=rows)
+def oracle_fwd(q, k, v, causal, scale, heads, rows=None, window=(-1, -1)):
+    kv = kv_heads(q, k, heads)
+    return oracle.attn_fwd(heads_f64(q, heads), heads_f64(k, kv), heads_f64(v, kv), causal=causal,
+                           scale=scale, rows=rows, window=window)
+
+
+def oracle_bwd(q, k, v, do, causal, scale, heads, rows=None, window=(-1, -1)):
+    kv = kv_heads(q, k, heads)
+    return oracle.attn_bwd(heads_f64(q, heads), heads_f64(k, kv), heads_f64(v, kv), heads_f64(do, heads),
+                           causal=causal, scale=scale, rows=rows, window=window)
+
+
+def oracle_bwd_grouped(q, k, v, do, causal, scale, b, h_kv, window=(-1, -1)):
+    """dQ of the whole group of query heads of K/V head (b, h_kv), and that K/V head's dK/dV summed over the
+    group (the oracle's grouped-head path)."""
+    group = q.shape[2] // k.shape[2]
+    qh = [(b, h_kv * group + g) for g in range(group)]
+    return oracle.attn_bwd(heads_f64(q, qh), heads_f64(k, [(b, h_kv)]), heads_f64(v, [(b, h_kv)]),
+                           heads_f64(do, qh), causal=causal, scale=scale, window=window)
 
 
 def gather_rows(x, heads, rows=None):
