@@ -22,7 +22,7 @@ FA_F16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
                 -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
-EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
            "fa_status_string", "fa_device_status")
 
 _lib = None
@@ -52,6 +52,8 @@ def lib():
     L.fa_bwd_stage.argtypes = [i] + L.fa_bwd.argtypes
     L.fa_fwd_ex.restype = i
     L.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp]
+    L.fa_fwd_fp8.restype = i
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, f, f, f, vp]
     L.fa_bwd_ex.restype = i
     L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_bwd_workspace_size.restype = sz
@@ -111,6 +113,34 @@ def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, wind
                          _dtype_code(q), _stream_ptr(stream))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_ex")
+    return out, lse
+
+
+def fwd_fp8(q, k, v, causal=False, scale=None, descale=(1.0, 1.0, 1.0), out=None, lse=None, stream=None,
+            window=(-1, -1)):
+    """Forward attention on float8_e4m3fn inputs (D = 128). The real inputs are q * descale[0], k * descale[1],
+    v * descale[2]. Returns (out bf16 [B,Sq,H,D], lse fp32 [B,H,Sq])."""
+    import torch
+
+    dev = q.device
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_bshd(n, t, dev)
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError("%s must be float8_e4m3fn, got %s" % (n, t.dtype))
+    B, Sq, H, D = q.shape
+    Sk = k.shape[1]
+    if out is None:
+        out = torch.empty((B, Sq, H, D), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bfloat16")
+    rc = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H,
+                          k.shape[2], D, int(bool(causal)), int(window[0]), int(window[1]),
+                          float(0.0 if scale is None else scale), float(descale[0]), float(descale[1]),
+                          float(descale[2]), _stream_ptr(stream))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_fwd_fp8")
     return out, lse
 
 

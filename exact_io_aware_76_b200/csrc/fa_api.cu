@@ -70,15 +70,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B, S, H, D] 16-bit tensor; box = 64 head-dim elements (one 128-byte swizzle row) x 1 head x `rows` rows.
+// [B, S, H, D] tensor of 16-bit (dtype FA_F16/FA_BF16) or 8-bit (dtype -1: e4m3 bytes) elements; box = one
+// 128-byte swizzle row of head-dim elements x 1 head x `rows` rows.
+constexpr int kDtypeE4M3 = -1;
 int make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D, int dtype, int rows) {
   auto enc = encode_fn();
   if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t es = dtype == kDtypeE4M3 ? 1 : 2;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es, (cuuint64_t)S * H * D * es};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1, (cuuint32_t)rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+  const CUtensorMapDataType t = dtype == kDtypeE4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                : dtype == FA_BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(m, t, 4,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -97,15 +103,16 @@ int check_common(int B, int Sq, int Sk, int H, int D, float scale, int dtype) {
   return FA_OK;
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool FP8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p, int dev,
                cudaStream_t stream) {
+  using L = FwdSmem<D, FP8>;
   static bool attr_done[kMaxDevices] = {};
-  auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL>;
-  int rc = ensure_smem_attr(kern, FwdSmem<D>::kAlloc, dev, attr_done);
+  auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, FP8>;
+  int rc = ensure_smem_attr(kern, L::kAlloc, dev, attr_done);
   if (rc) return rc;
   const unsigned grid = (unsigned)(p.n_qblk * p.B * p.H);
-  kern<<<grid, FwdSmem<D>::kThreads, FwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, p);
+  kern<<<grid, L::kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -233,12 +240,53 @@ int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse
   // Head-major CTA order once a head's re-read K/V no longer fit in L2 together with the other heads'.
   p.head_major = (2.0 * B * Sk * Hkv * D * 2 > kHeadMajorBytes) ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
+  p.v_descale = 1.f;
   const bool c = causal != 0;
   if (D == 64)
     return dtype == FA_BF16 ? dispatch_fwd_causal<64, true>(c, tq, tk, tv, p, dev, stream)
                             : dispatch_fwd_causal<64, false>(c, tq, tk, tv, p, dev, stream);
   return dtype == FA_BF16 ? dispatch_fwd_causal<128, true>(c, tq, tk, tv, p, dev, stream)
                           : dispatch_fwd_causal<128, false>(c, tq, tk, tv, p, dev, stream);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
+               int Hkv, int D, int causal, int window_left, int window_right, float scale, float q_descale,
+               float k_descale, float v_descale, cudaStream_t stream) {
+  if (!q || !k || !v || !out || !lse) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return FA_ERR_INVALID;
+  if (Hkv < 1 || H < 1 || H % Hkv != 0) return FA_ERR_INVALID;
+  if (!isfinite(q_descale) || !isfinite(k_descale) || !isfinite(v_descale) || q_descale <= 0.f ||
+      k_descale <= 0.f || v_descale <= 0.f)
+    return FA_ERR_INVALID;
+  int rc = check_common(B, Sq, Sk, H, D, scale, FA_BF16);
+  if (rc) return rc;
+  if (D != 128) return FA_ERR_UNSUPPORTED;  // an e4m3 row of 64 elements is only 64 bytes
+  int dev = 0;
+  if ((rc = current_device(&dev))) return rc;
+  if (scale == 0.f) scale = 1.f / sqrtf((float)D);
+
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_bshd_map(&tq, q, B, Sq, H, D, kDtypeE4M3, 128))) return rc;
+  if ((rc = make_bshd_map(&tk, k, B, Sk, Hkv, D, kDtypeE4M3, 128))) return rc;
+  if ((rc = make_bshd_map(&tv, v, B, Sk, Hkv, D, kDtypeE4M3, 128))) return rc;
+  FwdParams p;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.group = H / Hkv;
+  p.win_left = window_left < 0 ? -1 : window_left;
+  p.win_right = window_right < 0 ? -1 : window_right;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.n_qblk = (Sq + 255) / 256;
+  p.n_kv_total = (Sk + 127) / 128;
+  p.head_major = (2.0 * B * Sk * Hkv * D > kHeadMajorBytes) ? 1 : 0;
+  p.scale_log2 = scale * q_descale * k_descale * fa::kLog2e;
+  p.v_descale = v_descale;
+  return causal ? launch_fwd<128, true, true, true>(tq, tk, tv, p, dev, stream)
+                : launch_fwd<128, true, false, true>(tq, tk, tv, p, dev, stream);
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H, int D,

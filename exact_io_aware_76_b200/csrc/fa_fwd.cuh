@@ -44,15 +44,21 @@ struct FwdParams {
   int n_qblk;      // ceil(Sq / 256)
   int n_kv_total;  // ceil(Sk / 128)
   int head_major;  // CTA order: 1 = all query blocks of a head together (K/V reuse in L2), 0 = heavy-first
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (8-bit inputs: times the q and k descale factors)
+  float v_descale;   // 8-bit inputs: O is multiplied by this (1 otherwise)
 };
 
-template <int D>
+// kFP8: e4m3 inputs (the FP8 forward of the skill page's Workflow 3), one byte per element.
+template <int D, bool kFP8 = false>
 struct FwdSmem {
   static constexpr int kBM = 128, kBN = 128, kNQ = 2;
-  static constexpr int kChunks = D / 64;              // 128-byte column chunks per row
-  static constexpr int kTileBytes = 128 * D * 2;      // one 128-row tile of 16-bit values
-  static constexpr int kStages = (D == 128) ? 2 : 4;  // K/V ring depth
+  static constexpr int kElem = kFP8 ? 1 : 2;                      // bytes per input element
+  static constexpr int kChunks = D * kElem / 128;                 // 128-byte column chunks per row
+  static constexpr int kChunkElems = 128 / kElem;                 // elements per 128-byte chunk
+  static constexpr int kTileBytes = 128 * D * kElem;              // one 128-row tile
+  static constexpr int kStages = (kTileBytes >= 32768) ? 2 : 4;   // K/V ring depth
+  static constexpr int kKSteps = D * kElem / 32;                  // MMA steps over the head dim (32 B each)
+  static constexpr int kPCols = kFP8 ? 32 : 64;                   // TMEM columns of a packed P row
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kNQ * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
@@ -67,11 +73,12 @@ struct FwdSmem {
   static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
 };
 
-template <int D, bool kBF16, bool kCausal>
+// kBF16: the 16-bit input type (and output type); with kFP8 the inputs are e4m3 and the output is bf16.
+template <int D, bool kBF16, bool kCausal, bool kFP8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdSmem<D>;
+  using L = FwdSmem<D, kFP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
@@ -173,7 +180,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < 2; ++t) {
         if (n_kv[t] == 0) continue;
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kQOff + t * L::kTileBytes + c * 16384, &tm_q, q_full, 64 * c, h,
+          tma_load_4d(smem + L::kQOff + t * L::kTileBytes + c * 16384, &tm_q, q_full, L::kChunkElems * c, h,
                       qblk * 256 + t * 128, b);
       }
       int j = 0;  // index into the CTA's key tiles; the key tile is j_begin + j
@@ -183,10 +190,12 @@ __global__ void __launch_bounds__(384, 1)
         if (j >= L::kStages && !mbar_wait(&kv_empty[s], ((j / L::kStages) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kKOff + s * L::kTileBytes + c * 16384, &tm_k, &k_full[s], 64 * c, h_kv, key0, b);
+          tma_load_4d(smem + L::kKOff + s * L::kTileBytes + c * 16384, &tm_k, &k_full[s], L::kChunkElems * c, h_kv,
+                      key0, b);
         mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kVOff + s * L::kTileBytes + c * 16384, &tm_v, &v_full[s], 64 * c, h_kv, key0, b);
+          tma_load_4d(smem + L::kVOff + s * L::kTileBytes + c * 16384, &tm_v, &v_full[s], L::kChunkElems * c, h_kv,
+                      key0, b);
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA exits (bounded; own flag, not the CTA's).
@@ -204,33 +213,42 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_iter > 0) {
-      constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, D, false, true);
+      constexpr uint32_t idesc_qk = kFP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(kBF16, 128, 128, false, false);
+      constexpr uint32_t idesc_pv = kFP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(kBF16, 128, D, false, true);
       // Base descriptors are built once; every MMA below adds a compile-time byte offset to one of them
       // (building a descriptor per instruction would make this single issuing thread the bottleneck).
       const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
       const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
       const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kVOff), 16384, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      // S_t = Q_t K_j^T : K-major A and B, K (= head dim) advanced 16 elements (32 B) per instruction.
+      // S_t = Q_t K_j^T : K-major A and B, K (= head dim) advanced 32 B per instruction (16 bf16/fp16 or 32
+      // e4m3 elements).
       auto issue_qk = [&](int t, int s) {
         const uint32_t s_tmem = tmem + t * 128;
         const uint64_t a0 = sdesc_add(q_desc, t * L::kTileBytes), b0 = sdesc_add(k_desc, s * L::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::kKSteps; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-          umma_ss(s_tmem, sdesc_add(a0, koff), sdesc_add(b0, koff), idesc_qk, kk > 0 ? 1u : 0u);
+          if (kFP8)
+            umma_ss_f8(s_tmem, sdesc_add(a0, koff), sdesc_add(b0, koff), idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(s_tmem, sdesc_add(a0, koff), sdesc_add(b0, koff), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t V_j : A = P_t from TMEM (16 keys = 8 columns per instruction), B = V_j MN-major
-      // (16 keys = 16 rows of 128 B = 2048 B per instruction; 64-wide head-dim blocks 16 KB apart).
+      // O_t += P_t V_j : A = P_t from TMEM (8 columns per instruction: 16 keys of 16-bit P, or 32 keys of e4m3
+      // P), B = V_j MN-major (as many 128-byte key rows per instruction; 64-wide head-dim blocks 16 KB apart).
       auto issue_pv = [&](int t, int s, bool acc) {
         const uint32_t o_tmem = tmem + 256 + t * D;
         const uint32_t p_tmem = tmem + t * 128;
         const uint64_t b0 = sdesc_add(v_desc, s * L::kTileBytes);
+        constexpr int kKeys = kFP8 ? 32 : 16;  // keys per instruction
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          umma_ts(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * 2048), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 128 / kKeys; ++kk) {
+          if (kFP8)
+            umma_ts_f8(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * kKeys * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          else
+            umma_ts(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * kKeys * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       // Key tile jj (local index j = jj - j_begin) serves Q tile t when j_lo[t] <= jj < j_lo[t] + n_kv[t]; a
       // tile's first S is issued when the walk reaches its interval, every later one right after its PV.
@@ -333,16 +351,26 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
       float sum = 0.f;
-      uint32_t pk[64];
+      uint32_t pk[L::kPCols];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
+      for (int c = 0; c < 128; c += 4) {
         const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
         const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
-        sum += p0 + p1;
-        pk[c / 2] = pack2<kBF16>(p0, p1);
+        const float p2 = ex2_approx(fmaf(s[c + 2], p.scale_log2, -m_use));
+        const float p3 = ex2_approx(fmaf(s[c + 3], p.scale_log2, -m_use));
+        sum += (p0 + p1) + (p2 + p3);
+        if (kFP8) {
+          pk[c / 4] = pack4_e4m3(p0, p1, p2, p3);
+        } else {
+          pk[c / 2] = pack2<kBF16>(p0, p1);
+          pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+        }
       }
       l += sum;
-      tmem_st_x64(s_tmem, pk);
+      if (kFP8)
+        tmem_st_x32(s_tmem, pk);
+      else
+        tmem_st_x64(s_tmem, pk);
       tmem_st_wait();
       tc_fence_before_sync();
       mbar_arrive(&p_full[t]);
@@ -352,7 +380,7 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after_sync();
       const bool valid_row = row < p.Sq;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f) ? p.v_descale / l : 0.f;
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {

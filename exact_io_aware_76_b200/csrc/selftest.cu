@@ -144,14 +144,16 @@ __global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns, int* w
 //   shape 3: SS, A MN-major, B MN-major  4: TS, B K-major               5: SS, A MN-major, B K-major
 // MN-major operands use the 128-byte swizzle (the only form the kernels use).
 __global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int shape, int N, int iters, int swz,
-                                                                     long long* cycles) {
+                                                                     long long* cycles, const uint8_t* src) {
   using namespace fa;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 196608);  // operands read at most 192 KB
   uint32_t* holder = reinterpret_cast<uint32_t*>(smem + 196608 + 48);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 196608 + 52);
+  volatile int* stop = reinterpret_cast<volatile int*>(smem + 196608 + 56);
   if (threadIdx.x == 0) {
+    *stop = 0;
     for (int i = 0; i < 5; ++i) mbar_init(bar + i, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -164,6 +166,28 @@ __global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int shape, in
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *holder;
+  // Shapes 9 and 10 replay shape 8 while other warps add traffic: 9 = one thread streams 16 KB bulk copies from
+  // global memory into spare shared memory [200 KB, 216 KB); 10 = warps 2-3 stream TMEM loads/stores on the spare
+  // columns 448-511 of their lanes. Both stop when the MMA thread is done (or after a fixed number of rounds).
+  if (shape == 9 && threadIdx.x == 32) {
+    uint64_t* lbar = bar + 4;
+    int drain = 0;
+    for (int r = 0; r < 200000 && !*stop; ++r) {
+      mbar_arrive_expect_tx(lbar, 16384);
+      bulk_load(smem + 204800, src + (size_t)(r & 63) * 16384, 16384, lbar);
+      if (!mbar_wait(lbar, r & 1, &drain)) break;
+    }
+  }
+  if (shape == 10 && (threadIdx.x >> 5) >= 2) {
+    const uint32_t lane_base = tmem + (((threadIdx.x >> 5) * 32) << 16);
+    uint32_t rr[32];
+    for (int i = 0; i < 32; ++i) rr[i] = i;
+    for (int r = 0; r < 200000 && !*stop; ++r) {
+      tmem_ld_x32(lane_base + 448 + (r & 1) * 32, rr);
+      tmem_st_x32(lane_base + 448 + ((r + 1) & 1) * 32, rr);
+      tmem_st_wait();
+    }
+  }
   if (threadIdx.x == 0) {
     const uint32_t a = smem_u32(smem), b = smem_u32(smem + 32768);
     // shape: 0 SS A-K B-K, 1 SS A-K B-MN, 2 TS B-MN, 3 SS A-MN B-MN, 4 TS B-K, 5 SS A-MN B-K.
@@ -179,7 +203,7 @@ __global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int shape, in
       ad[kk] = a_mn ? sdesc_sw128(a + kk * 2048, 16384, 1024) : sdesc_sw128(a + (kk % 4) * 32, 16, 1024);
     }
     const long long t0 = clock64();
-    if (shape == 8) {
+    if (shape >= 8) {
       // Same sequence on the kernel's own layout: K [0,32K), V [32K,64K), Q stages [64K,112K), dO stages
       // [112K,160K), dS^T buffers [160K,192K); tiles rotate through the stages.
       const uint32_t base = smem_u32(smem);
@@ -250,12 +274,97 @@ __global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int shape, in
     umma_commit(bar);
     mbar_wait(bar, 0, abort_flag);
     cycles[blockIdx.x] = clock64() - t0;
+    *stop = 1;
   }
   tc_fence_before_sync();
   __syncthreads();
   if (threadIdx.x < 32) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// 8-bit (e4m3) products with K = 128: variant 0: A [128][128] K-major, B [N][128] K-major (the S = Q K^T
+// form); variant 1: A [128][128] placed in TMEM four elements per column, B [128][N] MN-major (the O = P V form).
+__global__ void __launch_bounds__(128, 1)
+    selftest_f8_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                       const uint8_t* a_glob, float* c, int variant, int N) {
+  using namespace fa;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + 16384;
+  uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + 32768);
+  uint64_t* bar_mma = bar_load + 1;
+  uint32_t* holder = reinterpret_cast<uint32_t*>(smem + 32768 + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 32768 + 20);
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(holder, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *holder;  // C at [0, N), A (variant 1) at [128, 160)
+  if (threadIdx.x == 0) {
+    uint32_t bytes = N * 128;
+    if (variant == 0) {
+      tma_load_2d(sa, &ta, bar_load, 0, 0);
+      bytes += 128 * 128;
+    }
+    tma_load_2d(sb, &tb, bar_load, 0, 0);
+    mbar_arrive_expect_tx(bar_load, bytes);
+  }
+  if (variant == 1) {
+    const uint32_t lane_base = tmem + ((warp * 32) << 16);
+    const int m = threadIdx.x;
+    uint32_t r[32];
+    for (int i = 0; i < 32; ++i)
+      r[i] = a_glob[m * 128 + 4 * i] | (a_glob[m * 128 + 4 * i + 1] << 8) | (a_glob[m * 128 + 4 * i + 2] << 16) |
+             (static_cast<uint32_t>(a_glob[m * 128 + 4 * i + 3]) << 24);
+    tmem_st_x32(lane_base + 128, r);
+    tmem_st_wait();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (threadIdx.x == 0) {
+    bool ok = mbar_wait(bar_load, 0, abort_flag);
+    tc_fence_after_sync();
+    const uint32_t a_base = smem_u32(sa), b_base = smem_u32(sb);
+    const uint32_t idesc = idesc_e4m3(128, N, false, variant == 1);
+    for (int kk = 0; ok && kk < 4; ++kk) {
+      if (variant == 0)
+        umma_ss_f8(tmem, sdesc_sw128(a_base + kk * 32, 16, 1024), sdesc_sw128(b_base + kk * 32, 16, 1024), idesc, kk > 0);
+      else
+        umma_ts_f8(tmem, tmem + 128 + kk * 8, sdesc_sw128(b_base + kk * 4096, 16384, 1024), idesc, kk > 0);
+    }
+    umma_commit(bar_mma);
+  }
+  __syncwarp();
+  bool ok = mbar_wait(bar_mma, 0, abort_flag);
+  tc_fence_after_sync();
+  if (ok) {
+    const uint32_t lane_base = tmem + ((warp * 32) << 16);
+    const int m = warp * 32 + lane;
+    for (int n0 = 0; n0 < N; n0 += 32) {
+      float r[32];
+      tmem_ld_x32(lane_base + n0, reinterpret_cast<uint32_t*>(r));
+      for (int i = 0; i < 32; ++i) c[m * N + n0 + i] = r[i];
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -331,16 +440,59 @@ extern "C" __attribute__((visibility("default"))) int fa_selftest_wait_timeout(u
 // Runs the throughput probe on `ctas` CTAs (one per SM) and copies the per-CTA cycle counts to cycles_host.
 extern "C" __attribute__((visibility("default"))) int fa_selftest_mma_rate(int shape, int N, int iters, int swz,
                                                                             int ctas, long long* cycles_host) {
-  if (shape < 0 || shape > 8 || (N != 64 && N != 128 && N != 256) || iters < 32 || (iters % 32) != 0 || ctas < 1 ||
+  if (shape < 0 || shape > 10 || (N != 64 && N != 128 && N != 256) || iters < 32 || (iters % 32) != 0 || ctas < 1 ||
       ctas > 1024 || swz != 128)
     return -1;
   long long* d = nullptr;
+  uint8_t* src = nullptr;
   if (cudaMalloc(&d, sizeof(long long) * ctas) != cudaSuccess) return -3;
-  const int smem = 196608 + 64 + 1024;  // > half the SM's shared memory: one CTA per SM
+  if (cudaMalloc(&src, 64 * 16384) != cudaSuccess) return -3;
+  cudaMemset(src, 0, 64 * 16384);
+  const int smem = 221184 + 1024;  // operands up to 192 KB, bookkeeping at 192 KB, bulk-copy target 200-216 KB  // > half the SM's shared memory: one CTA per SM
   cudaFuncSetAttribute(selftest_mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  selftest_mma_rate_kernel<<<ctas, 128, smem>>>(shape, N, iters, swz, d);
+  selftest_mma_rate_kernel<<<ctas, 128, smem>>>(shape, N, iters, swz, d, src);
   if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return -3;
   cudaMemcpy(cycles_host, d, sizeof(long long) * ctas, cudaMemcpyDeviceToHost);
   cudaFree(d);
+  cudaFree(src);
   return 0;
+}
+
+// 8-bit layout check: variant 0 C = A B^T with A [128][128], B [N][128]; variant 1 C = A B with A [128][128]
+// (through TMEM), B [128][N]; all e4m3 bytes. N in {64, 128}.
+extern "C" __attribute__((visibility("default"))) int fa_selftest_f8(int variant, const void* a, const void* b,
+                                                                      float* c, int N) {
+  if ((variant != 0 && variant != 1) || (N != 64 && N != 128) || !a || !b || !c) return -1;
+  auto enc = encode_fn();
+  if (!enc) return -3;
+  CUtensorMap ta, tb;
+  const cuuint32_t es[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {128, 128};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, 128};
+    if (enc(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return -3;
+  }
+  {
+    // variant 0: B [N][128] rows of 128 bytes; variant 1: B [128][N]: for N = 64 the rows are 64 bytes, so the
+    // box takes the full 128-byte swizzle row only when N = 128.
+    const cuuint64_t dims[2] = {variant == 0 ? 128u : (cuuint64_t)N, variant == 0 ? (cuuint64_t)N : 128u};
+    const cuuint64_t strides[1] = {variant == 0 ? 128u : (cuuint64_t)N};
+    const cuuint32_t box[2] = {variant == 0 ? 128u : (cuuint32_t)N, variant == 0 ? (cuuint32_t)N : 128u};
+    if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(b), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return -3;
+  }
+  const int smem = 32768 + 64 + 1024;
+  cudaFuncSetAttribute(selftest_f8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  selftest_f8_kernel<<<1, 128, smem>>>(ta, tb, (const uint8_t*)a, c, variant, N);
+  if (cudaGetLastError() != cudaSuccess) return -3;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -3;
+  int st = 0;
+  cudaMemcpyFromSymbol(&st, fa::g_device_status, sizeof(int));
+  return st;
 }

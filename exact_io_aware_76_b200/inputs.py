@@ -36,3 +36,17 @@ def make_inputs(B, Sq, Sk, H, D, dtype, seed, sigma=1.0, device="cuda", with_dou
     do = draw((B, Sq, H, D), dtype, g, device, 1.0)
     return q, k, v, do
 
+
+def draw_e4m3(shape, generator, device, sigma=1.0, per_tensor_scale=False):
+    """One N(0,1)*sigma float32 tensor stored as float8_e4m3fn plus its descale factor, the FP8 input form of
+    the skill page's Workflow 3. Without ``per_tensor_scale`` the samples are rounded to e4m3 directly (descale
+    1); with it they are first divided by amax/448 so that the largest magnitude lands on e4m3's largest
+    finite value (448), and the descale is amax/448. The real input is ``x_e4m3 * descale``."""
+    x = torch.randn(shape, generator=generator, device=device, dtype=torch.float32)
+    if sigma != 1.0:
+        x.mul_(sigma)
+    descale = 1.0
+    if per_tensor_scale:
+        descale = float(x.abs().max()) / 448.0
+        x.div_(descale)
+    return x.to(torch.float8_e4m3fn), descale

@@ -78,3 +78,20 @@ def test_bwd_workspace_checks():
 def test_workspace_size_invalid_is_zero():
     assert fa.workspace_size(0, 128, 1, 64) == 0
     assert fa.workspace_size(1, 128, 1, 96) == 0
+
+
+def fwd_fp8_call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Sq=128, Sk=128, H=2, Hkv=1, D=128, causal=0,
+                 left=-1, right=-1, scale=0.0, qd=1.0, kd=1.0, vd=1.0):
+    return fa.lib().fa_fwd_fp8(q, k, v, o, lse, B, Sq, Sk, H, Hkv, D, causal, left, right, scale, qd, kd, vd, None)
+
+
+@pytest.mark.parametrize("kw", [dict(q=None), dict(v=MISALIGNED), dict(lse=None), dict(Hkv=0), dict(Hkv=3),
+                                dict(B=0), dict(Sq=0), dict(scale=float("nan")), dict(qd=0.0), dict(kd=-1.0),
+                                dict(vd=float("inf")), dict(qd=float("nan"))])
+def test_fwd_fp8_rejects_invalid(kw):
+    assert fwd_fp8_call(**kw) == -1
+
+
+@pytest.mark.parametrize("D", [32, 64, 256])
+def test_fwd_fp8_unsupported_head_dim(D):
+    assert fwd_fp8_call(D=D) == -2

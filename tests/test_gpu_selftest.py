@@ -72,3 +72,23 @@ def test_bounded_wait_gives_up_and_reports_timeout(st):
     out, lse = fa.fwd(q, q, q)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all() and fa.device_status() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant,N", [(0, 64), (0, 128), (1, 128)])
+def test_e4m3_layouts(st, variant, N):
+    """8-bit (e4m3) tcgen05 products: the S = Q K^T form from shared memory, and the O = P V form with A in TMEM
+    (four consecutive K elements per 32-bit column) and an MN-major B."""
+    st.fa_selftest_f8.restype = ctypes.c_int
+    st.fa_selftest_f8.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77 + variant + N)
+    a = (torch.randn(128, 128, device="cuda", generator=g) * 2).to(torch.float8_e4m3fn)
+    b = (torch.randn(N, 128, device="cuda", generator=g) * 2).to(torch.float8_e4m3fn) if variant == 0 else \
+        (torch.randn(128, N, device="cuda", generator=g) * 2).to(torch.float8_e4m3fn)
+    c = torch.full((128, N), float("nan"), device="cuda", dtype=torch.float32)
+    rc = st.fa_selftest_f8(variant, a.view(torch.uint8).data_ptr(), b.view(torch.uint8).data_ptr(), c.data_ptr(), N)
+    assert rc == 0, rc
+    ref = a.double() @ (b.double().t() if variant == 0 else b.double())
+    err = (c.double() - ref).abs().max().item()
+    assert err <= 1e-3 * max(1.0, ref.abs().max().item()), err
