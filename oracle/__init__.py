@@ -13,6 +13,8 @@ Array convention (numpy, float64, C-contiguous), one entry per attention head:
     q, dout: [n_q_heads, Sq, D]    k, v: [n_kv_heads, Sk, D]   (q head h reads K/V head h // (n_q / n_kv))
     rows:    [n_q_heads, n_rows] int64 query rows to evaluate (default: all rows)
     window:  (left, right) sliding window around the key aligned with each query; -1 = unbounded side
+    dropout: (dropout_p, seed, offset) attention dropout with a Philox4x32-10 mask (None = no dropout);
+             head_index[h] is listed head h's head number b * H + h in the mask's counter (default: h)
 Outputs:
     fwd -> out [n_q_heads, n_rows, D], lse [n_q_heads, n_rows]   (natural-log LSE, scale included)
     bwd -> dq [n_q_heads, n_rows, D], dk/dv [n_kv_heads, Sk, D] (contributions of the listed rows, summed
@@ -53,6 +55,18 @@ class Oracle:
         lib.oracle_attn_bwd.restype = ctypes.c_int
         lib.oracle_attn_bwd.argtypes = [_F64P, _F64P, _F64P, _F64P, i64, i64, i64, i64, i64, ctypes.c_int, i64,
                                         i64, ctypes.c_double, _I64P, i64, _F64P, _F64P, _F64P]
+        u32, u64, dbl = ctypes.c_uint32, ctypes.c_uint64, ctypes.c_double
+        lib.oracle_attn_fwd_dropout.restype = ctypes.c_int
+        lib.oracle_attn_fwd_dropout.argtypes = [_F64P, _F64P, _F64P, i64, i64, i64, i64, i64, ctypes.c_int, i64, i64,
+                                                dbl, dbl, u64, u32, _I64P, _I64P, i64, _F64P, _F64P]
+        lib.oracle_attn_bwd_dropout.restype = ctypes.c_int
+        lib.oracle_attn_bwd_dropout.argtypes = [_F64P, _F64P, _F64P, _F64P, i64, i64, i64, i64, i64, ctypes.c_int,
+                                                i64, i64, dbl, dbl, u64, u32, _I64P, _I64P, i64, _F64P, _F64P,
+                                                _F64P]
+        lib.oracle_philox4x32_10.restype = None
+        lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32), ctypes.POINTER(u32)]
+        lib.oracle_dropout_mask.restype = ctypes.c_int
+        lib.oracle_dropout_mask.argtypes = [dbl, u64, u32, i64, i64, i64, ctypes.POINTER(ctypes.c_uint8)]
         self.lib = lib
 
     @staticmethod
@@ -73,7 +87,33 @@ class Oracle:
             raise ValueError("rows must be [n_heads, n_rows]")
         return q, k, v, rows
 
-    def fwd(self, q, k, v, causal=False, scale=None, rows=None, window=(-1, -1)):
+    @staticmethod
+    def _heads(head_index, nh):
+        if head_index is None:
+            head_index = np.arange(nh, dtype=np.int64)
+        head_index = np.ascontiguousarray(head_index, dtype=np.int64)
+        if head_index.shape != (nh,):
+            raise ValueError("head_index must have one entry per q head")
+        return head_index
+
+    def philox4x32_10(self, ctr, key):
+        """Philox4x32-10 of one 4-word counter under a 2-word key (both unsigned 32-bit words)."""
+        c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+        kk = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        out = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, kk, out)
+        return [int(x) for x in out]
+
+    def dropout_mask(self, dropout_p, seed, offset, bh, Sq, Sk):
+        """Keep mask (bool [Sq, Sk]) of head number bh."""
+        keep = np.zeros((Sq, Sk), np.uint8)
+        rc = self.lib.oracle_dropout_mask(float(dropout_p), int(seed), int(offset), int(bh), int(Sq), int(Sk),
+                                          keep.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        if rc != 0:
+            raise ValueError("oracle_dropout_mask rejected its arguments")
+        return keep.astype(bool)
+
+    def fwd(self, q, k, v, causal=False, scale=None, rows=None, window=(-1, -1), dropout=None, head_index=None):
         q, k, v, rows = self._prep(q, k, v, rows)
         nh, Sq, D = q.shape
         nkv, Sk = k.shape[0], k.shape[1]
@@ -82,16 +122,26 @@ class Oracle:
         nr = rows.shape[1]
         out = np.zeros((nh, nr, D), np.float64)
         lse = np.zeros((nh, nr), np.float64)
-        rc = self.lib.oracle_attn_fwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P), v.ctypes.data_as(_F64P),
-                                      nh, nkv, Sq, Sk, D, int(bool(causal)), int(window[0]), int(window[1]),
-                                      float(scale),
-                                      rows.ctypes.data_as(_I64P), nr, out.ctypes.data_as(_F64P),
-                                      lse.ctypes.data_as(_F64P))
+        if dropout is None:
+            rc = self.lib.oracle_attn_fwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P),
+                                          v.ctypes.data_as(_F64P), nh, nkv, Sq, Sk, D, int(bool(causal)),
+                                          int(window[0]), int(window[1]), float(scale),
+                                          rows.ctypes.data_as(_I64P), nr, out.ctypes.data_as(_F64P),
+                                          lse.ctypes.data_as(_F64P))
+        else:
+            hi = self._heads(head_index, nh)
+            rc = self.lib.oracle_attn_fwd_dropout(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P),
+                                                  v.ctypes.data_as(_F64P), nh, nkv, Sq, Sk, D, int(bool(causal)),
+                                                  int(window[0]), int(window[1]), float(scale),
+                                                  float(dropout[0]), int(dropout[1]), int(dropout[2]),
+                                                  hi.ctypes.data_as(_I64P), rows.ctypes.data_as(_I64P), nr,
+                                                  out.ctypes.data_as(_F64P), lse.ctypes.data_as(_F64P))
         if rc != 0:
             raise ValueError("oracle_attn_fwd rejected its arguments")
         return out, lse
 
-    def bwd(self, q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1)):
+    def bwd(self, q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1), dropout=None,
+            head_index=None):
         q, k, v, rows = self._prep(q, k, v, rows)
         dout = np.ascontiguousarray(dout, dtype=np.float64)
         if dout.shape != q.shape:
@@ -104,11 +154,21 @@ class Oracle:
         dq = np.zeros((nh, nr, D), np.float64)
         dk = np.zeros((nkv, Sk, D), np.float64)
         dv = np.zeros((nkv, Sk, D), np.float64)
-        rc = self.lib.oracle_attn_bwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P), v.ctypes.data_as(_F64P),
-                                      dout.ctypes.data_as(_F64P), nh, nkv, Sq, Sk, D, int(bool(causal)),
-                                      int(window[0]), int(window[1]), float(scale),
-                                      rows.ctypes.data_as(_I64P), nr, dq.ctypes.data_as(_F64P),
-                                      dk.ctypes.data_as(_F64P), dv.ctypes.data_as(_F64P))
+        if dropout is None:
+            rc = self.lib.oracle_attn_bwd(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P),
+                                          v.ctypes.data_as(_F64P), dout.ctypes.data_as(_F64P), nh, nkv, Sq, Sk, D,
+                                          int(bool(causal)), int(window[0]), int(window[1]), float(scale),
+                                          rows.ctypes.data_as(_I64P), nr, dq.ctypes.data_as(_F64P),
+                                          dk.ctypes.data_as(_F64P), dv.ctypes.data_as(_F64P))
+        else:
+            hi = self._heads(head_index, nh)
+            rc = self.lib.oracle_attn_bwd_dropout(q.ctypes.data_as(_F64P), k.ctypes.data_as(_F64P),
+                                                  v.ctypes.data_as(_F64P), dout.ctypes.data_as(_F64P), nh, nkv, Sq,
+                                                  Sk, D, int(bool(causal)), int(window[0]), int(window[1]),
+                                                  float(scale), float(dropout[0]), int(dropout[1]),
+                                                  int(dropout[2]), hi.ctypes.data_as(_I64P),
+                                                  rows.ctypes.data_as(_I64P), nr, dq.ctypes.data_as(_F64P),
+                                                  dk.ctypes.data_as(_F64P), dv.ctypes.data_as(_F64P))
         if rc != 0:
             raise ValueError("oracle_attn_bwd rejected its arguments")
         return dq, dk, dv
@@ -124,14 +184,24 @@ def _get():
     return _default
 
 
-def attn_fwd(q, k, v, causal=False, scale=None, rows=None, window=(-1, -1)):
+def attn_fwd(q, k, v, causal=False, scale=None, rows=None, window=(-1, -1), dropout=None, head_index=None):
     """O and LSE of the listed query rows (all rows by default). See the module docstring for layouts."""
-    return _get().fwd(q, k, v, causal=causal, scale=scale, rows=rows, window=window)
+    return _get().fwd(q, k, v, causal=causal, scale=scale, rows=rows, window=window, dropout=dropout,
+                      head_index=head_index)
 
 
-def attn_bwd(q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1)):
+def attn_bwd(q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1), dropout=None, head_index=None):
     """dQ of the listed rows and their dK/dV contributions. See the module docstring for layouts."""
-    return _get().bwd(q, k, v, dout, causal=causal, scale=scale, rows=rows, window=window)
+    return _get().bwd(q, k, v, dout, causal=causal, scale=scale, rows=rows, window=window, dropout=dropout,
+                      head_index=head_index)
+
+
+def philox4x32_10(ctr, key):
+    return _get().philox4x32_10(ctr, key)
+
+
+def dropout_mask(dropout_p, seed, offset, bh, Sq, Sk):
+    return _get().dropout_mask(dropout_p, seed, offset, bh, Sq, Sk)
 
 
 def bshd_heads(x, b, h):

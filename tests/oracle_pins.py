@@ -20,7 +20,12 @@ What pins it:
   * grouped K/V heads (skill page, Workflow 2 Step 3): the same as repeating each K/V head over its group
     (dK/dV summed over the group), finite differences through the shared heads, and torch SDPA with
     enable_gqa; the sliding window (Workflow 2 Steps 2-3, window_size=(left, right)): a window wider than the
-    sequence changes nothing, (0, 0) keeps only the aligned key, finite differences, SDPA with a band mask.
+    sequence changes nothing, (0, 0) keeps only the aligned key, finite differences, SDPA with a band mask;
+  * dropout (the dropout_p argument of the skill page's call): Philox4x32-10 against its published
+    known-answer vectors and a keep block derived by hand from one of them (tests/golden/philox_dropout.json);
+    dropout_p = 0 is the plain path; the keep rate matches 1 - t/256; O averaged over many seeds converges to
+    the undropped O (the 1/(1 - p) rescale) with LSE unchanged; with V = I the output is P o Z itself; finite
+    differences with the mask held fixed.
 """
 import json
 import math
@@ -387,7 +392,132 @@ def pin_window_gqa_sdpa_crosscheck(orc):
             _close(dv, tv.grad[0].numpy(), what="SDPA GQA/window dV")
 
 
+def _golden_philox():
+    with open(os.path.join(HERE, "golden", "philox_dropout.json")) as f:
+        return json.load(f)
+
+
+def pin_philox_known_answers(orc):
+    g = _golden_philox()
+    for case in g["philox4x32_10"]:
+        ctr = [int(x, 16) for x in case["ctr"]]
+        key = [int(x, 16) for x in case["key"]]
+        out = orc.philox4x32_10(ctr, key)
+        assert out == [int(x, 16) for x in case["out"]], ("Philox4x32-10 known answer", case["ctr"], out)
+
+
+def pin_dropout_keep_block(orc):
+    kb = _golden_philox()["keep_block"]
+    keep = orc.dropout_mask(kb["dropout_p"], kb["seed"], kb["offset"], kb["bh"], 4, 4)
+    assert np.array_equal(keep, np.array(kb["keep"], bool)), ("hand-derived keep block", keep.astype(int))
+
+
+def pin_dropout_zero_is_plain(orc):
+    r = _rng(16)
+    q, k, v, do = (r.standard_normal((2, 7, 3)) for _ in range(4))
+    for causal in (False, True):
+        o1, l1 = orc.fwd(q, k, v, causal=causal, scale=0.6)
+        o2, l2 = orc.fwd(q, k, v, causal=causal, scale=0.6, dropout=(0.0, 99, 3))
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2), "dropout_p = 0 changes the forward"
+        g1 = orc.bwd(q, k, v, do, causal=causal, scale=0.6)
+        g2 = orc.bwd(q, k, v, do, causal=causal, scale=0.6, dropout=(0.0, 99, 3))
+        for a, b in zip(g1, g2):
+            assert np.array_equal(a, b), "dropout_p = 0 changes the backward"
+
+
+def pin_dropout_keep_rate(orc):
+    # keep fraction of a 256 x 512 mask within 5 binomial standard deviations of 1 - t/256, for several p;
+    # two different seeds, offsets or head numbers agree only as often as independent masks would
+    n = 256 * 512
+    for p in (0.1, 0.3, 0.5, 0.9):
+        t = math.floor(256 * p + 0.5)
+        keep_p = 1 - t / 256
+        m = orc.dropout_mask(p, 1234, 7, 3, 256, 512)
+        assert abs(m.mean() - keep_p) <= 5 * math.sqrt(keep_p * (1 - keep_p) / n), ("keep rate", p, m.mean())
+        agree_p = keep_p ** 2 + (1 - keep_p) ** 2
+        for other in (orc.dropout_mask(p, 1235, 7, 3, 256, 512), orc.dropout_mask(p, 1234, 8, 3, 256, 512),
+                      orc.dropout_mask(p, 1234, 7, 4, 256, 512)):
+            agree = (m == other).mean()
+            assert abs(agree - agree_p) <= 5 * math.sqrt(agree_p * (1 - agree_p) / n), ("independent masks", p)
+
+
+def pin_dropout_unbiased(orc):
+    # E_seed[O_dropout] = O: each kept probability is scaled by 1 / (1 - p'); LSE ignores dropout
+    r = _rng(17)
+    q, k, v = (r.standard_normal((1, 3, 2)) for _ in range(3))
+    p = 0.25
+    pe = math.floor(256 * p + 0.5) / 256
+    o_ref, l_ref = orc.fwd(q, k, v, scale=0.9)
+    n = 3000
+    acc = np.zeros_like(o_ref)
+    for seed in range(n):
+        o, l = orc.fwd(q, k, v, scale=0.9, dropout=(p, seed, 0))
+        assert np.array_equal(l, l_ref), "LSE depends on dropout"
+        acc += o
+    # variance of one O element: sum_j P_ij^2 v_jd^2 p'/(1-p') <= sum_j P_ij v_jd^2 p'/(1-p'), the latter being
+    # the plain forward with V replaced by v_jd^2
+    var = np.zeros_like(o_ref)
+    for d in range(2):
+        vd = np.zeros((1, 3, 2))
+        vd[0, :, 0] = v[0, :, d] ** 2
+        od, _ = orc.fwd(q, k, vd, scale=0.9)
+        var[0, :, d] = od[0, :, 0] * pe / (1 - pe)
+    tol = 6 * np.sqrt(np.maximum(var, 0.0) / n) + 1e-12
+    assert np.all(np.abs(acc / n - o_ref) <= tol), ("dropout mean", np.abs(acc / n - o_ref).max(), tol.max())
+
+
+def pin_dropout_identity_values(orc):
+    # With Sk = D and V = I, O = (P o Z) itself: P from the plain forward, Z from the exported mask
+    r = _rng(18)
+    Sq, Sk = 9, 6
+    q = r.standard_normal((2, Sq, Sk))
+    k = r.standard_normal((2, Sk, Sk))
+    eye = np.broadcast_to(np.eye(Sk), (2, Sk, Sk)).copy()
+    p = 0.3
+    pe = math.floor(256 * p + 0.5) / 256
+    for causal in (False, True):
+        P, _ = orc.fwd(q, k, eye, causal=causal, scale=0.5)
+        heads = np.array([5, 11])
+        O, _ = orc.fwd(q, k, eye, causal=causal, scale=0.5, dropout=(p, 42, 9), head_index=heads)
+        for h in range(2):
+            keep = orc.dropout_mask(p, 42, 9, heads[h], Sq, Sk)
+            _close(O[h], P[h] * keep / (1 - pe), what="O = P o Z with V = I")
+
+
+def pin_dropout_finite_differences(orc):
+    r = _rng(19)
+    h = 1e-6
+    for (nq, nkv, Sq, Sk, D, causal, window, p) in ((2, 1, 5, 6, 2, False, (-1, -1), 0.3),
+                                                     (2, 2, 6, 6, 3, True, (2, 0), 0.5)):
+        q = r.standard_normal((nq, Sq, D))
+        k = r.standard_normal((nkv, Sk, D))
+        v = r.standard_normal((nkv, Sk, D))
+        do = r.standard_normal((nq, Sq, D))
+        drop = (p, 77, 1)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.7, window=window, dropout=drop)
+
+        def loss(qq, kk, vv):
+            out, _ = orc.fwd(qq, kk, vv, causal=causal, scale=0.7, window=window, dropout=drop)
+            return float(np.sum(out * do))
+
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                args = {"q": q, "k": k, "v": v}
+                xp = x.copy()
+                xp[idx] += h
+                xm = x.copy()
+                xm[idx] -= h
+                ap = dict(args, **{name: xp})
+                am = dict(args, **{name: xm})
+                num[idx] = (loss(ap["q"], ap["k"], ap["v"]) - loss(am["q"], am["k"], am["v"])) / (2 * h)
+            err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+            assert err <= 1e-6, ("dropout finite differences d" + name, err)
+
+
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
-            pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck]
+            pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,
+            pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_zero_is_plain, pin_dropout_keep_rate,
+            pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences]

@@ -95,3 +95,20 @@ def test_fwd_fp8_rejects_invalid(kw):
 @pytest.mark.parametrize("D", [32, 64, 256])
 def test_fwd_fp8_unsupported_head_dim(D):
     assert fwd_fp8_call(D=D) == -2
+
+
+def fwd_drop_call(p, B=1, Sq=128, Sk=128, H=1, Hkv=1, D=64):
+    return fa.lib().fa_fwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, B, Sq, Sk, H, Hkv, D, 0, -1, -1, 0.0, 0, p, 1, 0, None)
+
+
+@pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, 0.999, float("nan"), float("inf")])
+def test_dropout_rejects_bad_probability(p):
+    # 0.999 rounds to t = 256 (everything dropped): rejected like p >= 1
+    assert fwd_drop_call(p) == -1
+    assert fa.lib().fa_bwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, 1, 1, 64, 0, -1,
+                                   -1, 0.0, 0, p, 1, 0, FAKE, 1 << 30, None) == -1
+
+
+def test_dropout_rejects_bad_shapes_first():
+    assert fwd_drop_call(0.1, B=0) == -1
+    assert fwd_drop_call(0.1, D=96) == -2

@@ -24,15 +24,24 @@ MUTANTS = {
                           "const double *kh = k + (h % n_kv_heads) * Sk * D;\n            const double *vh = v + (h % n_kv_heads) * Sk * D;"),
     "gqa_dk_not_summed": ("dkh[j * D + d] += scale * gk;", "dkh[j * D + d] = scale * gk;"),
     "lse_drops_max": ("double lse = m + log(sum);", "double lse = log(sum);"),
-    "output_uses_k": ("o[d] += p[j] * vh[j * D + d];", "o[d] += p[j] * kh[j * D + d];"),
+    "output_uses_k": ("o[d] += pz * vh[j * D + d];", "o[d] += pz * kh[j * D + d];"),
     "dp_uses_k": ("acc += doh[i * D + d] * vh[j * D + d];", "acc += doh[i * D + d] * kh[j * D + d];"),
     "ds_sign": ("dSi[j] = Pi[j] * (dP[j] - Di);", "dSi[j] = Pi[j] * (dP[j] + Di);"),
     "drop_Di": ("Di += Pi[j] * dP[j];", "Di += 0.0 * dP[j];"),
     "dq_no_scale": ("for (int64_t d = 0; d < D; ++d) dqi[d] *= scale;", ""),
     "dq_uses_v": ("dqi[d] += dSi[j] * kh[j * D + d];", "dqi[d] += dSi[j] * vh[j * D + d];"),
     "dk_uses_dout": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * doh[i * D + d];"),
-    "dv_uses_dS": ("gv += P[r * Sk + j] * doh[i * D + d];", "gv += dS[r * Sk + j] * doh[i * D + d];"),
+    "dv_uses_dS": ("gv += G[r * Sk + j] * doh[i * D + d];", "gv += dS[r * Sk + j] * doh[i * D + d];"),
     "dk_no_scale": ("dkh[j * D + d] += scale * gk;", "dkh[j * D + d] += gk;"),
+    "philox_no_key_bump": ("k0 += PHILOX_W0;", ""),
+    "philox_swapped_products": ("uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;", "uint32_t n0 = (uint32_t)(p0 >> 32) ^ c1 ^ k0;"),
+    "dropout_word_byte_swapped": ("uint32_t byte = (w[i & 3] >> (8 * (j & 3))) & 0xffu;",
+                                  "uint32_t byte = (w[j & 3] >> (8 * (i & 3))) & 0xffu;"),
+    "dropout_threshold_flipped": ("return byte >= (uint32_t)dr->t ?", "return byte < (uint32_t)dr->t ?"),
+    "dropout_no_rescale": ("? 1.0 / (1.0 - dr->t / 256.0) : 0.0;", "? 1.0 : 0.0;"),
+    "dropout_counter_ignores_head": ("(uint32_t)(j >> 2), (uint32_t)bh, dr->offset};", "(uint32_t)(j >> 2), 0u, dr->offset};"),
+    "dropout_dv_undropped": ("gv += G[r * Sk + j] * doh[i * D + d];", "gv += P[r * Sk + j] * doh[i * D + d];"),
+    "dropout_dp_unmasked": ("dP[j] = z * acc;", "dP[j] = acc;"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
