@@ -22,7 +22,7 @@ FA_F16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
                 -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
-EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
            "fa_status_string", "fa_device_status")
 
 _lib = None
@@ -54,6 +54,12 @@ def lib():
     L.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp]
     L.fa_fwd_fp8.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, f, f, f, vp]
+    u32, u64 = ctypes.c_uint32, ctypes.c_uint64
+    L.fa_fwd_dropout.restype = i
+    L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, f, u64, u32, vp]
+    L.fa_bwd_dropout.restype = i
+    L.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, f, u64, u32,
+                                 vp, sz, vp]
     L.fa_bwd_ex.restype = i
     L.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_bwd_workspace_size.restype = sz
@@ -94,8 +100,12 @@ def _check_bshd(name, t, dev):
         raise ValueError("%s must be a contiguous [B, S, H, D] tensor" % name)
 
 
-def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, window=(-1, -1)):
-    """Forward attention. Returns (out [B,Sq,H,D] in q's dtype, lse fp32 [B,H,Sq])."""
+def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, window=(-1, -1), dropout_p=0.0, seed=0,
+        offset=0):
+    """Forward attention. Returns (out [B,Sq,H,D] in q's dtype, lse fp32 [B,H,Sq]).
+
+    ``dropout_p`` > 0 drops attention probabilities with the Philox mask of ``fa_fwd_dropout`` (include/fa.h),
+    keyed by ``seed`` (64-bit) and ``offset`` (32-bit); the backward must get the same three values."""
     import torch
 
     dev = q.device
@@ -108,11 +118,14 @@ def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, wind
     if lse is None:
         lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
     Hkv = k.shape[2]
-    rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, Hkv,
-                         D, int(bool(causal)), int(window[0]), int(window[1]), float(0.0 if scale is None else scale),
-                         _dtype_code(q), _stream_ptr(stream))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, Hkv, D,
+            int(bool(causal)), int(window[0]), int(window[1]), float(0.0 if scale is None else scale), _dtype_code(q))
+    if dropout_p:
+        rc = lib().fa_fwd_dropout(*args, float(dropout_p), int(seed), int(offset), _stream_ptr(stream))
+    else:
+        rc = lib().fa_fwd_ex(*args, _stream_ptr(stream))
     if rc != FA_OK:
-        raise FAError(rc, "fa_fwd_ex")
+        raise FAError(rc, "fa_fwd_dropout" if dropout_p else "fa_fwd_ex")
     return out, lse
 
 
@@ -149,7 +162,7 @@ def workspace_size(B, Sq, H, D):
 
 
 def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None,
-        stage=-1, window=(-1, -1)):
+        stage=-1, window=(-1, -1), dropout_p=0.0, seed=0, offset=0):
     """Backward attention (P recomputed from lse). Returns (dq, dk, dv) in q's dtype.
 
     ``stage`` selects one of the three launches (0 preprocess, 1 main, 2 dQ conversion; -1 all), see
@@ -170,7 +183,14 @@ def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=
     Hkv = k.shape[2]
     sc = float(0.0 if scale is None else scale)
     ws_args = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
-    if stage == -1:
+    if dropout_p:
+        if stage != -1:
+            raise ValueError("single backward stages are available for plain attention only")
+        rc = lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, Hkv, D,
+                                  int(bool(causal)), int(window[0]), int(window[1]), sc, _dtype_code(q),
+                                  float(dropout_p), int(seed), int(offset), *ws_args)
+    elif stage == -1:
         rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, Hkv, D, int(bool(causal)),
                              int(window[0]), int(window[1]), sc, _dtype_code(q), *ws_args)

@@ -103,12 +103,12 @@ int check_common(int B, int Sq, int Sk, int H, int D, float scale, int dtype) {
   return FA_OK;
 }
 
-template <int D, bool BF16, bool CAUSAL, bool FP8 = false>
+template <int D, bool BF16, bool CAUSAL, bool FP8 = false, bool DROP = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p, int dev,
                cudaStream_t stream) {
   using L = FwdSmem<D, FP8>;
   static bool attr_done[kMaxDevices] = {};
-  auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, FP8>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, CAUSAL, FP8, DROP>;
   int rc = ensure_smem_attr(kern, L::kAlloc, dev, attr_done);
   if (rc) return rc;
   const unsigned grid = (unsigned)(p.n_qblk * p.B * p.H);
@@ -119,6 +119,9 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 template <int D, bool BF16>
 int dispatch_fwd_causal(bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const FwdParams& p, int dev, cudaStream_t s) {
+  if (p.drop_t != 0)
+    return causal ? launch_fwd<D, BF16, true, false, true>(tq, tk, tv, p, dev, s)
+                  : launch_fwd<D, BF16, false, false, true>(tq, tk, tv, p, dev, s);
   return causal ? launch_fwd<D, BF16, true>(tq, tk, tv, p, dev, s) : launch_fwd<D, BF16, false>(tq, tk, tv, p, dev, s);
 }
 
@@ -150,11 +153,11 @@ int grid_for(long long work, int per_block, int dev) {
 }
 
 // stage -1: all three launches; 0: preprocess; 1: main; 2: dQ conversion.
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool DROP = false>
 int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t stream) {
   static bool attr_done[kMaxDevices] = {};
-  auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL>;
+  auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL, DROP>;
   int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
   if (rc) return rc;
   if (stage < 0 || stage == 0) {
@@ -177,6 +180,9 @@ int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CU
 template <int D, bool BF16>
 int dispatch_bwd_causal(int stage, bool causal, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t s) {
+  if (p.drop_t != 0)
+    return causal ? launch_bwd<D, BF16, true, true>(stage, tq, tk, tv, tdo, p, dev, s)
+                  : launch_bwd<D, BF16, false, true>(stage, tq, tk, tv, tdo, p, dev, s);
   return causal ? launch_bwd<D, BF16, true>(stage, tq, tk, tv, tdo, p, dev, s)
                 : launch_bwd<D, BF16, false>(stage, tq, tk, tv, tdo, p, dev, s);
 }
@@ -208,9 +214,22 @@ int fa_device_status(int reset) {
   return v;
 }
 
-int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
-              int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
-              cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+// Dropout threshold t = floor(256 p + 1/2); -1 unless 0 <= p < 1 and t <= 255.
+int dropout_threshold(float p) {
+  if (!(p >= 0.f && p < 1.f)) return -1;
+  const int t = (int)floorf(256.f * p + 0.5f);
+  return t <= 255 ? t : -1;
+}
+}  // namespace
+
+static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
+                    int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+                    float dropout_p, uint64_t seed, uint32_t offset, cudaStream_t stream) {
+  const int drop_t = dropout_threshold(dropout_p);
+  if (drop_t < 0) return FA_ERR_INVALID;
   if (!q || !k || !v || !out || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return FA_ERR_INVALID;
   if (Hkv < 1 || H < 1 || H % Hkv != 0) return FA_ERR_INVALID;
@@ -240,13 +259,33 @@ int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse
   // Head-major CTA order once a head's re-read K/V no longer fit in L2 together with the other heads'.
   p.head_major = (2.0 * B * Sk * Hkv * D * 2 > kHeadMajorBytes) ? 1 : 0;
   p.scale_log2 = scale * fa::kLog2e;
-  p.v_descale = 1.f;
+  p.drop_t = (uint32_t)drop_t;
+  p.drop_k0 = (uint32_t)seed;
+  p.drop_k1 = (uint32_t)(seed >> 32);
+  p.drop_off = offset;
+  p.v_descale = 1.f / (1.f - drop_t / 256.f);
   const bool c = causal != 0;
   if (D == 64)
     return dtype == FA_BF16 ? dispatch_fwd_causal<64, true>(c, tq, tk, tv, p, dev, stream)
                             : dispatch_fwd_causal<64, false>(c, tq, tk, tv, p, dev, stream);
   return dtype == FA_BF16 ? dispatch_fwd_causal<128, true>(c, tq, tk, tv, p, dev, stream)
                           : dispatch_fwd_causal<128, false>(c, tq, tk, tv, p, dev, stream);
+}
+
+extern "C" {
+
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
+              int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+              cudaStream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Sq, Sk, H, Hkv, D, causal, window_left, window_right, scale, dtype, 0.f, 0,
+                  0, stream);
+}
+
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
+                   int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+                   float dropout_p, uint64_t seed, uint32_t offset, cudaStream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Sq, Sk, H, Hkv, D, causal, window_left, window_right, scale, dtype,
+                  dropout_p, seed, offset, stream);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk, int H,
@@ -285,6 +324,8 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* ls
   p.head_major = (2.0 * B * Sk * Hkv * D > kHeadMajorBytes) ? 1 : 0;
   p.scale_log2 = scale * q_descale * k_descale * fa::kLog2e;
   p.v_descale = v_descale;
+  p.drop_t = 0;
+  p.drop_k0 = p.drop_k1 = p.drop_off = 0;
   return causal ? launch_fwd<128, true, true, true>(tq, tk, tv, p, dev, stream)
                 : launch_fwd<128, true, false, true>(tq, tk, tv, p, dev, stream);
 }
@@ -301,9 +342,11 @@ size_t fa_bwd_workspace_size(int B, int Sq, int H, int D) {
 
 static int bwd_impl(int stage, const void* q, const void* k, const void* v, const void* out, const float* lse,
                     const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D,
-                    int causal, int window_left, int window_right, float scale, int dtype, void* workspace,
-                    size_t workspace_bytes, cudaStream_t stream) {
+                    int causal, int window_left, int window_right, float scale, int dtype, float dropout_p,
+                    uint64_t seed, uint32_t offset, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (stage < -1 || stage > 2) return FA_ERR_INVALID;
+  const int drop_t = dropout_threshold(dropout_p);
+  if (drop_t < 0) return FA_ERR_INVALID;
   if (Hkv < 1 || H < 1 || H % Hkv != 0) return FA_ERR_INVALID;
   const void* ptrs[9] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* ptr : ptrs)
@@ -348,6 +391,11 @@ static int bwd_impl(int stage, const void* q, const void* k, const void* v, cons
   p.head_major = ((double)B * Sq * H * D * 8 > kHeadMajorBytes) ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * fa::kLog2e;
+  p.drop_t = (uint32_t)drop_t;
+  p.drop_k0 = (uint32_t)seed;
+  p.drop_k1 = (uint32_t)(seed >> 32);
+  p.drop_off = offset;
+  p.drop_scale = 1.f / (1.f - drop_t / 256.f);
   const bool c = causal != 0;
   if (D == 64)
     return dtype == FA_BF16 ? dispatch_bwd_causal<64, true>(stage, c, tq, tk, tv, tdo, p, dev, stream)
@@ -360,7 +408,7 @@ int fa_bwd_stage(int stage, const void* q, const void* k, const void* v, const v
                  const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int D, int causal,
                  float scale, int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return bwd_impl(stage, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, H, D, causal, -1, -1, scale, dtype,
-                  workspace, workspace_bytes, stream);
+                  0.f, 0, 0, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
@@ -368,7 +416,15 @@ int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, cons
               int window_right, float scale, int dtype, void* workspace, size_t workspace_bytes,
               cudaStream_t stream) {
   return bwd_impl(-1, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, Hkv, D, causal, window_left, window_right,
-                  scale, dtype, workspace, workspace_bytes, stream);
+                  scale, dtype, 0.f, 0, 0, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D, int causal,
+                   int window_left, int window_right, float scale, int dtype, float dropout_p, uint64_t seed,
+                   uint32_t offset, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_impl(-1, q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, Hkv, D, causal, window_left, window_right,
+                  scale, dtype, dropout_p, seed, offset, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout, void* dq,
@@ -411,7 +467,6 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
   if (fa_bwd_workspace_size(B, Sq, H, D) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
   int dev = 0;
   if ((rc = current_device(&dev))) return rc;
-  if (rc) return rc;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(dev, &scratch))) return rc;
   return fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Sq, Sk, H, D, causal, scale, dtype, scratch,

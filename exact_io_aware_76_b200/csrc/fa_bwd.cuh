@@ -30,6 +30,7 @@
 // the dQ partial landing in the S^T columns that the dV product has already read.
 // Query tile BQ = 64 rows for D = 128 and 128 rows for D = 64, so that every MMA has M = 128.
 #pragma once
+#include "dropout.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -50,6 +51,14 @@ struct BwdParams {
   int n_kblk;        // ceil(Sk / 128)
   int head_major;    // CTA order: 1 = all key tiles of a head together (L2 reuse), 0 = heavy-first
   float scale, scale_log2;
+  uint32_t drop_t;                      // dropout threshold t (0 = no dropout)
+  uint32_t drop_k0, drop_k1, drop_off;  // Philox key (seed) and counter word 3 (offset)
+  float drop_scale;                     // 1 / (1 - t/256)
+};
+
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
 };
 
 constexpr float kLog2eB = 1.4426950408889634f;
@@ -165,7 +174,8 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // Pipeline (NB = 2): the MMA thread issues S^T/dP^T of tile it+2 right after dV/dK/dQ of tile it, so the
 // compute warps work on tile it+1 while the tensor core runs both. Buffers are indexed by it % NB, stages
 // of the Q/dO ring by it % NQS; every barrier's phases are waited in order.
-template <int D, bool kBF16, bool kCausal>
+// kDrop: attention dropout; a separate instance so the plain path keeps its registers.
+template <int D, bool kBF16, bool kCausal, bool kDrop = false>
 __global__ void __launch_bounds__(384, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -378,8 +388,22 @@ __global__ void __launch_bounds__(384, 1)
       const int hi_c = has_left ? key - off + p.win_left - q0 : BQ;
       // Whole tile visible to every key of this CTA: no element mask.
       const bool need_mask = (has_right && key0 + 127 - off - right > q0) || (has_left && key0 - off + p.win_left < q0 + BQ - 1);
+      // One 64-query chunk; with dropout (kDrop) the mask's bytes for the chunk come first: per 16 queries the
+      // four lanes of this key's 4-key block each generate one 4x4 block, transpose its bytes (word = key) and
+      // exchange words, so that kw[c / 4] holds this key's bytes for queries c .. c + 3 of the chunk.
+      auto chunk = [&](int c0, auto drop_tag) {
+        constexpr bool kDrop = decltype(drop_tag)::value;
+        uint32_t kw[kDrop ? 16 : 1];
+        if constexpr (kDrop) {
+          const uint32_t bh = static_cast<uint32_t>(b * p.H + h_kv * p.group + it / n_q);
 #pragma unroll
-      for (int c0 = 0; c0 < BQ; c0 += 64) {
+          for (int g = 0; g < 4; ++g) {
+            philox4x32_10(static_cast<uint32_t>((q0 + c0 + 16 * g) >> 2) + (lane & 3u),
+                          static_cast<uint32_t>(key >> 2), bh, p.drop_off, p.drop_k0, p.drop_k1, kw + 4 * g);
+            byte_transpose4(kw + 4 * g);
+            quad_exchange(kw + 4 * g);
+          }
+        }
         float sv[64], dp[64];
         tmem_ld_x64_pair(lane_base + s_col + c0, reinterpret_cast<uint32_t*>(sv), lane_base + dp_col + c0,
                          reinterpret_cast<uint32_t*>(dp));
@@ -398,10 +422,24 @@ __global__ void __launch_bounds__(384, 1)
             if (c0 + c + 2 < lo_c || c0 + c + 2 > hi_c) p2 = 0.f;
             if (c0 + c + 3 < lo_c || c0 + c + 3 > hi_c) p3 = 0.f;
           }
-          pk[c / 2] = pack2<kBF16>(p0, p1);
-          pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
-          dk[c / 2] = pack2<kBF16>(p0 * (dp[c] - d4.x), p1 * (dp[c + 1] - d4.y));
-          dk[c / 2 + 1] = pack2<kBF16>(p2 * (dp[c + 2] - d4.z), p3 * (dp[c + 3] - d4.w));
+          if constexpr (kDrop) {
+            // dV takes the kept P (its 1/(1-t/256) is applied to dV at the end); dP reaching P is
+            // Z * (dO . v): 0 where dropped, scaled by 1/(1-t/256) where kept.
+            const uint32_t w = kw[c / 4];
+            const bool k0 = keep_byte(w, 0, p.drop_t), k1 = keep_byte(w, 1, p.drop_t);
+            const bool k2 = keep_byte(w, 2, p.drop_t), k3 = keep_byte(w, 3, p.drop_t);
+            const float z = p.drop_scale;
+            pk[c / 2] = pack2<kBF16>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
+            pk[c / 2 + 1] = pack2<kBF16>(k2 ? p2 : 0.f, k3 ? p3 : 0.f);
+            dk[c / 2] = pack2<kBF16>(p0 * ((k0 ? dp[c] * z : 0.f) - d4.x), p1 * ((k1 ? dp[c + 1] * z : 0.f) - d4.y));
+            dk[c / 2 + 1] = pack2<kBF16>(p2 * ((k2 ? dp[c + 2] * z : 0.f) - d4.z),
+                                         p3 * ((k3 ? dp[c + 3] * z : 0.f) - d4.w));
+          } else {
+            pk[c / 2] = pack2<kBF16>(p0, p1);
+            pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+            dk[c / 2] = pack2<kBF16>(p0 * (dp[c] - d4.x), p1 * (dp[c + 1] - d4.y));
+            dk[c / 2 + 1] = pack2<kBF16>(p2 * (dp[c + 2] - d4.z), p3 * (dp[c + 3] - d4.w));
+          }
         }
         tmem_st_x32(lane_base + s_col + c0 / 2, pk);
         // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
@@ -415,7 +453,9 @@ __global__ void __launch_bounds__(384, 1)
           const int unit = u ^ (j & 7);
           *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
-      }
+      };
+#pragma unroll
+      for (int c0 = 0; c0 < BQ; c0 += 64) chunk(c0, BoolTag<kDrop>{});
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before_sync();
@@ -430,7 +470,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         uint16_t* dst = reinterpret_cast<uint16_t*>(which == 0 ? p.dv : p.dk) + row_off;
-        const float mul = which == 0 ? 1.f : p.scale;
+        const float mul = which == 0 ? p.drop_scale : p.scale;
         const uint32_t col = which == 0 ? L::kColDV : L::kColDK;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {

@@ -27,6 +27,7 @@
 // factor 256); otherwise p is computed against the stale m. Both O and l use the same m, so the final
 // O/l is exact either way. LSE = (m + log2 l) * ln 2.
 #pragma once
+#include "dropout.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -45,7 +46,9 @@ struct FwdParams {
   int n_kv_total;  // ceil(Sk / 128)
   int head_major;  // CTA order: 1 = all query blocks of a head together (K/V reuse in L2), 0 = heavy-first
   float scale_log2;  // scale * log2(e) (8-bit inputs: times the q and k descale factors)
-  float v_descale;   // 8-bit inputs: O is multiplied by this (1 otherwise)
+  float v_descale;   // O is multiplied by this: the v descale of 8-bit inputs, 1 / (1 - t/256) with dropout
+  uint32_t drop_t;   // dropout threshold t (0 = no dropout; 16-bit inputs only)
+  uint32_t drop_k0, drop_k1, drop_off;  // Philox key (seed) and counter word 3 (offset)
 };
 
 // kFP8: e4m3 inputs (the FP8 forward of the skill page's Workflow 3), one byte per element.
@@ -74,7 +77,8 @@ struct FwdSmem {
 };
 
 // kBF16: the 16-bit input type (and output type); with kFP8 the inputs are e4m3 and the output is bf16.
-template <int D, bool kBF16, bool kCausal, bool kFP8 = false>
+// kDrop: attention dropout (16-bit inputs only); a separate instance so the plain path keeps its registers.
+template <int D, bool kBF16, bool kCausal, bool kFP8 = false, bool kDrop = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -352,18 +356,46 @@ __global__ void __launch_bounds__(384, 1)
       const float m_use = (m == -INFINITY) ? 0.f : m;
       float sum = 0.f;
       uint32_t pk[L::kPCols];
+      if constexpr (kDrop && !kFP8) {
+        // Dropout: P keeps only the kept probabilities (l sums them all; 1/(1-t/256) is applied to O at the
+        // end). Per 16 keys, the four lanes of this row's 4-row block each generate one 4x4 block of the mask
+        // and exchange words, so that w[k] holds this row's bytes for keys c16 + 4k .. c16 + 4k + 3.
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
-        const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
-        const float p2 = ex2_approx(fmaf(s[c + 2], p.scale_log2, -m_use));
-        const float p3 = ex2_approx(fmaf(s[c + 3], p.scale_log2, -m_use));
-        sum += (p0 + p1) + (p2 + p3);
-        if (kFP8) {
-          pk[c / 4] = pack4_e4m3(p0, p1, p2, p3);
-        } else {
-          pk[c / 2] = pack2<kBF16>(p0, p1);
-          pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+        for (int c16 = 0; c16 < 128; c16 += 16) {
+          uint32_t w[4];
+          philox4x32_10(static_cast<uint32_t>(row >> 2), static_cast<uint32_t>((key0 + c16) >> 2) + (lane & 3u),
+                        static_cast<uint32_t>(bh), p.drop_off, p.drop_k0, p.drop_k1, w);
+          quad_exchange(w);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int c = c16 + 4 * k;
+            float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
+            float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
+            float p2 = ex2_approx(fmaf(s[c + 2], p.scale_log2, -m_use));
+            float p3 = ex2_approx(fmaf(s[c + 3], p.scale_log2, -m_use));
+            sum += (p0 + p1) + (p2 + p3);
+            p0 = keep_byte(w[k], 0, p.drop_t) ? p0 : 0.f;
+            p1 = keep_byte(w[k], 1, p.drop_t) ? p1 : 0.f;
+            p2 = keep_byte(w[k], 2, p.drop_t) ? p2 : 0.f;
+            p3 = keep_byte(w[k], 3, p.drop_t) ? p3 : 0.f;
+            pk[c / 2] = pack2<kBF16>(p0, p1);
+            pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
+          const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
+          const float p2 = ex2_approx(fmaf(s[c + 2], p.scale_log2, -m_use));
+          const float p3 = ex2_approx(fmaf(s[c + 3], p.scale_log2, -m_use));
+          sum += (p0 + p1) + (p2 + p3);
+          if (kFP8) {
+            pk[c / 4] = pack4_e4m3(p0, p1, p2, p3);
+          } else {
+            pk[c / 2] = pack2<kBF16>(p0, p1);
+            pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+          }
         }
       }
       l += sum;

@@ -35,6 +35,7 @@
 #define FA_B200_H
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -84,6 +85,22 @@ FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, flo
                      cudaStream_t stream);
 
 /*
+ * Forward with attention dropout (the `dropout_p` argument of the skill page's flash_attn_func call, Workflow 2
+ * Step 2; the pages name it only). Arguments as fa_fwd_ex, plus:
+ *   dropout_p  drop probability, 0 <= dropout_p < 1; it is rounded to t / 256 with t = floor(256 p + 1/2), and
+ *              t = 256 is rejected (FA_ERR_INVALID).
+ *   seed       64-bit Philox4x32-10 key (low word, high word).
+ *   offset     32-bit counter word 3, so that successive calls with one seed draw different masks.
+ * Element (i, j) of head number bh = b * H + h is kept iff byte (j mod 4) of word (i mod 4) of
+ * Philox4x32-10(counter = (i / 4, j / 4, bh, offset), key = seed) is >= t. O = (P o Z) V with Z = keep / (1 -
+ * t / 256); LSE is that of the undropped scores, so fa_bwd_dropout with the same seed and offset regenerates the
+ * mask. dropout_p = 0 gives exactly fa_fwd_ex.
+ */
+FA_API int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                          int H, int Hkv, int D, int causal, int window_left, int window_right, float scale, int dtype,
+                          float dropout_p, uint64_t seed, uint32_t offset, cudaStream_t stream);
+
+/*
  * Forward on 8-bit inputs (the FP8 forward of the skill page's Workflow 3: "FP8 is a forward-only path, and the
  * input must be float8_e4m3fn"). q, k, v hold e4m3 bytes ([B,Sq,H,D] and [B,Sk,Hkv,D]); their real values are
  * the e4m3 values times q_descale, k_descale and v_descale (positive finite per-tensor factors; 1 for plain
@@ -94,6 +111,16 @@ FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, flo
 FA_API int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
                       int H, int Hkv, int D, int causal, int window_left, int window_right, float scale,
                       float q_descale, float k_descale, float v_descale, cudaStream_t stream);
+
+/*
+ * Backward of fa_fwd_dropout: arguments as fa_bwd_ex plus the forward's dropout_p, seed and offset (the same
+ * values, or the gradients are those of another mask). out must be the dropped output fa_fwd_dropout returned.
+ */
+FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int H, int Hkv, int D,
+                          int causal, int window_left, int window_right, float scale, int dtype, float dropout_p,
+                          uint64_t seed, uint32_t offset, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes (0 on invalid sizes). The workspace holds the fp32
