@@ -56,10 +56,6 @@ struct BwdParams {
   float drop_scale;                     // 1 / (1 - t/256)
 };
 
-template <bool B>
-struct BoolTag {
-  static constexpr bool value = B;
-};
 
 constexpr float kLog2eB = 1.4426950408889634f;
 

@@ -74,6 +74,10 @@ struct FwdSmem {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 384;
   static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
+  // One in kEmuEvery groups of four score columns computes its exponentials on the FMA pipe (0 = none).
+  // Measured on the GPT-shaped workload: with 8-bit inputs (half the MMA time per tile) one in four is
+  // fastest (+5%); with 16-bit inputs any share made the kernel slower, so none.
+  static constexpr int kEmuEvery = kFP8 ? 4 : 0;
 };
 
 // kBF16: the 16-bit input type (and output type); with kFP8 the inputs are e4m3 and the output is bf16.
@@ -329,9 +333,16 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 128; ++c)
           if (key0 + c < row_lo || key0 + c > row_hi) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // Row max: four independent chains of three-input maxima, then combined.
+      float mq[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int c = 4; c < 124; c += 8) {
+        mq[0] = fmax3(mq[0], s[c], s[c + 1]);
+        mq[1] = fmax3(mq[1], s[c + 2], s[c + 3]);
+        mq[2] = fmax3(mq[2], s[c + 4], s[c + 5]);
+        mq[3] = fmax3(mq[3], s[c + 6], s[c + 7]);
+      }
+      const float mx = fmaxf(fmax3(mq[0], mq[1], s[124]), fmax3(mq[2], mq[3], fmax3(s[125], s[126], s[127])));
       const float m_cand = fmaxf(m, mx * p.scale_log2);
       // Warp-uniform decision: TMEM loads/stores below are warp-collective.
       const bool rescale = __any_sync(0xffffffffu, m_cand > m + kRescaleLog2);
@@ -383,20 +394,46 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       } else {
+        // p = 2^(s * scale_log2 - m) with packed pairs for the FMA and the row sum. In a tile without an
+        // element mask every x is finite, and every kEmuEvery-th group of four columns takes its exponentials
+        // from the FMA pipe (exp2_poly2), which relieves the MUFU unit that otherwise bounds this loop.
+        auto p_loop = [&](auto emu_tag) {
+          constexpr bool kEmu = decltype(emu_tag)::value && L::kEmuEvery > 0;
+          const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m_use, -m_use);
+          uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_use));
-          const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_use));
-          const float p2 = ex2_approx(fmaf(s[c + 2], p.scale_log2, -m_use));
-          const float p3 = ex2_approx(fmaf(s[c + 3], p.scale_log2, -m_use));
-          sum += (p0 + p1) + (p2 + p3);
-          if (kFP8) {
-            pk[c / 4] = pack4_e4m3(p0, p1, p2, p3);
-          } else {
-            pk[c / 2] = pack2<kBF16>(p0, p1);
-            pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+          for (int c = 0; c < 128; c += 4) {
+            const uint64_t x01 = f2_fma(f2_pack(s[c], s[c + 1]), sc2, nm2);
+            const uint64_t x23 = f2_fma(f2_pack(s[c + 2], s[c + 3]), sc2, nm2);
+            float p0, p1, p2, p3;
+            if (kEmu && (c / 4) % L::kEmuEvery == L::kEmuEvery - 1) {
+              exp2_poly2(x01, p0, p1);
+              exp2_poly2(x23, p2, p3);
+            } else {
+              float a0, a1, a2, a3;
+              f2_unpack(x01, a0, a1);
+              f2_unpack(x23, a2, a3);
+              p0 = ex2_approx(a0);
+              p1 = ex2_approx(a1);
+              p2 = ex2_approx(a2);
+              p3 = ex2_approx(a3);
+            }
+            sum2 = f2_add(sum2, f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+            if (kFP8) {
+              pk[c / 4] = pack4_e4m3(p0, p1, p2, p3);
+            } else {
+              pk[c / 2] = pack2<kBF16>(p0, p1);
+              pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
+            }
           }
-        }
+          float s0, s1;
+          f2_unpack(sum2, s0, s1);
+          sum = s0 + s1;
+        };
+        if (need_mask)
+          p_loop(BoolTag<false>{});
+        else
+          p_loop(BoolTag<true>{});
       }
       l += sum;
       if (kFP8)

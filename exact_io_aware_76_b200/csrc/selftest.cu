@@ -496,3 +496,25 @@ extern "C" __attribute__((visibility("default"))) int fa_selftest_f8(int variant
   cudaMemcpyFromSymbol(&st, fa::g_device_status, sizeof(int));
   return st;
 }
+
+// ------------------------------------------------------------------------------------- exp2 on the FMA pipe
+// y[i] = exp2_poly2(x[i]) (pairs), z[i] = ex2.approx(x[i]): the softmax's two ways to exponentiate.
+__global__ void exp2_kernel(const float* x, float* y, float* z, int n_pairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pairs) return;
+  float y0, y1;
+  fa::exp2_poly2(fa::f2_pack(x[2 * i], x[2 * i + 1]), y0, y1);
+  y[2 * i] = y0;
+  y[2 * i + 1] = y1;
+  z[2 * i] = fa::ex2_approx(x[2 * i]);
+  z[2 * i + 1] = fa::ex2_approx(x[2 * i + 1]);
+}
+
+extern "C" __attribute__((visibility("default"))) int fa_selftest_exp2(const float* x, float* y, float* z, int n) {
+  if (n < 0 || (n & 1) || !x || !y || !z) return FA_ERR_INVALID;
+  if (n == 0) return FA_OK;
+  const int pairs = n / 2;
+  exp2_kernel<<<(pairs + 255) / 256, 256>>>(x, y, z, pairs);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}

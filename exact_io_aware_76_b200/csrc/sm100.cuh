@@ -278,6 +278,71 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// A compile-time flag as a type, for generic lambdas that instantiate one body twice.
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed pairs of fp32 (sm_100 executes add/fma on .f32x2 as one instruction for both halves).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// 2^x for a pair of values on the FMA pipe instead of the MUFU unit, for softmax elements that are finite and at
+// most a few units above 0. Range reduction: adding 1.5 * 2^23 rounds x (clamped to >= -125, so the result stays
+// a normal number) to the nearest integer n, held in the low mantissa bits of the sum; f = x - n lies in
+// [-1/2, 1/2]; 2^f comes from a degree-3 polynomial; n is then added into the exponent field. The polynomial's
+// coefficients minimise the maximum relative error of 2^f on [-1/2, 1/2] (fitted by Lawson's iteratively
+// reweighted least squares); that error is 8.4e-5, below half a unit of bf16 (2^-9) and of fp16 (2^-12).
+// A clamped input (x < -125) returns about 2^-125 instead of a smaller value or 0.
+__device__ __forceinline__ void exp2_poly2(uint64_t x, float& y0, float& y1) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  constexpr float kC0 = 0.999919593334198f, kC1 = 0.6932621598243713f, kC2 = 0.24271433055400848f,
+                  kC3 = 0.05521314591169357f;
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t shift = f2_pack(kShift, kShift);
+  const uint64_t t = f2_add(xc, shift);
+  const uint64_t f = f2_sub(xc, f2_sub(t, shift));
+  uint64_t q = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
+  q = f2_fma(q, f, f2_pack(kC1, kC1));
+  q = f2_fma(q, f, f2_pack(kC0, kC0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

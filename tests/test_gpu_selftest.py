@@ -92,3 +92,37 @@ def test_e4m3_layouts(st, variant, N):
     ref = a.double() @ (b.double().t() if variant == 0 else b.double())
     err = (c.double() - ref).abs().max().item()
     assert err <= 1e-3 * max(1.0, ref.abs().max().item()), err
+
+
+@pytest.mark.gpu
+def test_exp2_on_the_fma_pipe(st):
+    """The forward softmax computes some exponentials as exp2_poly2 (range reduction to the nearest integer
+    plus a degree-3 polynomial). Against fp64 exp2: relative error <= 1e-4 for x in [-125, 9] (the polynomial's
+    fitted bound is 8.4e-5, plus fp32 evaluation), about ex2.approx's own accuracy order; x below -125 returns at
+    most 2^-124 (a clamped, negligible weight); integers give exact powers of two up to the polynomial error."""
+    import numpy as np
+
+    st.fa_selftest_exp2.restype = ctypes.c_int
+    st.fa_selftest_exp2.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    x = torch.cat([torch.linspace(-125.0, 9.0, 1 << 20, device="cuda"),
+                   torch.rand(1 << 18, generator=g, device="cuda") * 134.0 - 125.0,
+                   torch.arange(-125, 10, device="cuda", dtype=torch.float32),
+                   torch.tensor([-0.5, 0.5, -0.49999997, 0.49999997, 0.0, -1e-30, 8.5], device="cuda"),
+                   torch.tensor([-126.0, -200.0, -1e30, -3e38], device="cuda")])
+    if x.numel() % 2:
+        x = torch.cat([x, torch.zeros(1, device="cuda")])
+    y = torch.empty_like(x)
+    z = torch.empty_like(x)
+    assert st.fa_selftest_exp2(x.data_ptr(), y.data_ptr(), z.data_ptr(), x.numel()) == 0
+    xs = x.cpu().double().numpy()
+    ys = y.cpu().double().numpy()
+    zs = z.cpu().double().numpy()
+    inside = xs >= -125.0
+    ref = np.exp2(xs[inside])
+    rel = np.abs(ys[inside] / ref - 1.0)
+    rel_mufu = np.abs(zs[inside] / ref - 1.0)
+    print("poly max rel %.3e, ex2.approx max rel %.3e" % (rel.max(), rel_mufu.max()))
+    assert rel.max() <= 1e-4
+    assert np.all((ys[~inside] > 0) & (ys[~inside] <= 2.0 ** -124))
