@@ -384,74 +384,109 @@ __global__ void __launch_bounds__(384, 1)
       const int hi_c = has_left ? key - off + p.win_left - q0 : BQ;
       // Whole tile visible to every key of this CTA: no element mask.
       const bool need_mask = (has_right && key0 + 127 - off - right > q0) || (has_left && key0 - off + p.win_left < q0 + BQ - 1);
-      // One 64-query chunk; with dropout (kDrop) the mask's bytes for the chunk come first: per 16 queries the
-      // four lanes of this key's 4-key block each generate one 4x4 block, transpose its bytes (word = key) and
-      // exchange words, so that kw[c / 4] holds this key's bytes for queries c .. c + 3 of the chunk.
-      auto chunk = [&](int c0, auto drop_tag) {
-        constexpr bool kDrop = decltype(drop_tag)::value;
-        uint32_t kw[kDrop ? 16 : 1];
-        if constexpr (kDrop) {
-          const uint32_t bh = static_cast<uint32_t>(b * p.H + h_kv * p.group + it / n_q);
+      if constexpr (kDrop) {
+        // One 64-query chunk; with dropout (kDrop) the mask's bytes for the chunk come first: per 16 queries the
+        // four lanes of this key's 4-key block each generate one 4x4 block, transpose its bytes (word = key) and
+        // exchange words, so that kw[c / 4] holds this key's bytes for queries c .. c + 3 of the chunk.
+        auto chunk = [&](int c0) {
+          uint32_t kw[16];
+          {
+            const uint32_t bh = static_cast<uint32_t>(b * p.H + h_kv * p.group + it / n_q);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            philox4x32_10(static_cast<uint32_t>((q0 + c0 + 16 * g) >> 2) + (lane & 3u),
-                          static_cast<uint32_t>(key >> 2), bh, p.drop_off, p.drop_k0, p.drop_k1, kw + 4 * g);
-            byte_transpose4(kw + 4 * g);
-            quad_exchange(kw + 4 * g);
+            for (int g = 0; g < 4; ++g) {
+              philox4x32_10(static_cast<uint32_t>((q0 + c0 + 16 * g) >> 2) + (lane & 3u),
+                            static_cast<uint32_t>(key >> 2), bh, p.drop_off, p.drop_k0, p.drop_k1, kw + 4 * g);
+              byte_transpose4(kw + 4 * g);
+              quad_exchange(kw + 4 * g);
+            }
           }
-        }
-        float sv[64], dp[64];
-        tmem_ld_x64_pair(lane_base + s_col + c0, reinterpret_cast<uint32_t*>(sv), lane_base + dp_col + c0,
-                         reinterpret_cast<uint32_t*>(dp));
-        uint32_t pk[32], dk[32];
+          float sv[64], dp[64];
+          tmem_ld_x64_pair(lane_base + s_col + c0, reinterpret_cast<uint32_t*>(sv), lane_base + dp_col + c0,
+                           reinterpret_cast<uint32_t*>(dp));
+          uint32_t pk[32], dk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
-          const float4 d4 = *reinterpret_cast<const float4*>(dvec + c0 + c);
-          float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -l4.x));
-          float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -l4.y));
-          float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l4.z));
-          float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l4.w));
-          if (need_mask) {
-            if (c0 + c < lo_c || c0 + c > hi_c) p0 = 0.f;
-            if (c0 + c + 1 < lo_c || c0 + c + 1 > hi_c) p1 = 0.f;
-            if (c0 + c + 2 < lo_c || c0 + c + 2 > hi_c) p2 = 0.f;
-            if (c0 + c + 3 < lo_c || c0 + c + 3 > hi_c) p3 = 0.f;
+          for (int c = 0; c < 64; c += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + c0 + c);
+            float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -l4.x));
+            float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -l4.y));
+            float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l4.z));
+            float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l4.w));
+            if (need_mask) {
+              if (c0 + c < lo_c || c0 + c > hi_c) p0 = 0.f;
+              if (c0 + c + 1 < lo_c || c0 + c + 1 > hi_c) p1 = 0.f;
+              if (c0 + c + 2 < lo_c || c0 + c + 2 > hi_c) p2 = 0.f;
+              if (c0 + c + 3 < lo_c || c0 + c + 3 > hi_c) p3 = 0.f;
+            }
+            {
+              // dV takes the kept P (its 1/(1-t/256) is applied to dV at the end); dP reaching P is
+              // Z * (dO . v): 0 where dropped, scaled by 1/(1-t/256) where kept.
+              const uint32_t w = kw[c / 4];
+              const bool k0 = keep_byte(w, 0, p.drop_t), k1 = keep_byte(w, 1, p.drop_t);
+              const bool k2 = keep_byte(w, 2, p.drop_t), k3 = keep_byte(w, 3, p.drop_t);
+              const float z = p.drop_scale;
+              pk[c / 2] = pack2<kBF16>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
+              pk[c / 2 + 1] = pack2<kBF16>(k2 ? p2 : 0.f, k3 ? p3 : 0.f);
+              dk[c / 2] = pack2<kBF16>(p0 * ((k0 ? dp[c] * z : 0.f) - d4.x), p1 * ((k1 ? dp[c + 1] * z : 0.f) - d4.y));
+              dk[c / 2 + 1] = pack2<kBF16>(p2 * ((k2 ? dp[c + 2] * z : 0.f) - d4.z),
+                                           p3 * ((k3 ? dp[c + 3] * z : 0.f) - d4.w));
+            }
           }
-          if constexpr (kDrop) {
-            // dV takes the kept P (its 1/(1-t/256) is applied to dV at the end); dP reaching P is
-            // Z * (dO . v): 0 where dropped, scaled by 1/(1-t/256) where kept.
-            const uint32_t w = kw[c / 4];
-            const bool k0 = keep_byte(w, 0, p.drop_t), k1 = keep_byte(w, 1, p.drop_t);
-            const bool k2 = keep_byte(w, 2, p.drop_t), k3 = keep_byte(w, 3, p.drop_t);
-            const float z = p.drop_scale;
-            pk[c / 2] = pack2<kBF16>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
-            pk[c / 2 + 1] = pack2<kBF16>(k2 ? p2 : 0.f, k3 ? p3 : 0.f);
-            dk[c / 2] = pack2<kBF16>(p0 * ((k0 ? dp[c] * z : 0.f) - d4.x), p1 * ((k1 ? dp[c + 1] * z : 0.f) - d4.y));
-            dk[c / 2 + 1] = pack2<kBF16>(p2 * ((k2 ? dp[c + 2] * z : 0.f) - d4.z),
-                                         p3 * ((k3 ? dp[c + 3] * z : 0.f) - d4.w));
-          } else {
+          tmem_st_x32(lane_base + s_col + c0 / 2, pk);
+          // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
+          // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The next tile's dP^T lands on these columns
+          // later, issued after the dK product, and the tensor core executes in issue order.
+          tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
+          // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
+          uint8_t* row = ds_row_base + (c0 / 64) * 16384;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int unit = u ^ (j & 7);
+            *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          }
+        };
+#pragma unroll
+        for (int c0 = 0; c0 < BQ; c0 += 64) chunk(c0);
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < BQ; c0 += 64) {
+          float sv[64], dp[64];
+          tmem_ld_x64_pair(lane_base + s_col + c0, reinterpret_cast<uint32_t*>(sv), lane_base + dp_col + c0,
+                           reinterpret_cast<uint32_t*>(dp));
+          uint32_t pk[32], dk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c0 + c);
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec + c0 + c);
+            float p0 = ex2_approx(fmaf(sv[c], p.scale_log2, -l4.x));
+            float p1 = ex2_approx(fmaf(sv[c + 1], p.scale_log2, -l4.y));
+            float p2 = ex2_approx(fmaf(sv[c + 2], p.scale_log2, -l4.z));
+            float p3 = ex2_approx(fmaf(sv[c + 3], p.scale_log2, -l4.w));
+            if (need_mask) {
+              if (c0 + c < lo_c || c0 + c > hi_c) p0 = 0.f;
+              if (c0 + c + 1 < lo_c || c0 + c + 1 > hi_c) p1 = 0.f;
+              if (c0 + c + 2 < lo_c || c0 + c + 2 > hi_c) p2 = 0.f;
+              if (c0 + c + 3 < lo_c || c0 + c + 3 > hi_c) p3 = 0.f;
+            }
             pk[c / 2] = pack2<kBF16>(p0, p1);
             pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
             dk[c / 2] = pack2<kBF16>(p0 * (dp[c] - d4.x), p1 * (dp[c + 1] - d4.y));
             dk[c / 2 + 1] = pack2<kBF16>(p2 * (dp[c + 2] - d4.z), p3 * (dp[c + 3] - d4.w));
           }
-        }
-        tmem_st_x32(lane_base + s_col + c0 / 2, pk);
-        // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
-        // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The next tile's dP^T lands on these columns
-        // later, issued after the dK product, and the tensor core executes in issue order.
-        tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
-        // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
-        uint8_t* row = ds_row_base + (c0 / 64) * 16384;
+          tmem_st_x32(lane_base + s_col + c0 / 2, pk);
+          // dS^T also goes to TMEM, into the dP^T columns already read (chunk c0 reads columns c0..c0+63 and
+          // writes c0/2..c0/2+31): the A operand of dK += dS^T Q. The next tile's dP^T lands on these columns
+          // later, issued after the dK product, and the tensor core executes in issue order.
+          tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
+          // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
+          uint8_t* row = ds_row_base + (c0 / 64) * 16384;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int unit = u ^ (j & 7);
-          *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          for (int u = 0; u < 8; ++u) {
+            const int unit = u ^ (j & 7);
+            *reinterpret_cast<uint4*>(row + unit * 16) = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          }
         }
-      };
-#pragma unroll
-      for (int c0 = 0; c0 < BQ; c0 += 64) chunk(c0, BoolTag<kDrop>{});
+      }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before_sync();
@@ -466,7 +501,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         uint16_t* dst = reinterpret_cast<uint16_t*>(which == 0 ? p.dv : p.dk) + row_off;
-        const float mul = which == 0 ? p.drop_scale : p.scale;
+        const float mul = which == 0 ? (kDrop ? p.drop_scale : 1.f) : p.scale;
         const uint32_t col = which == 0 ? L::kColDV : L::kColDK;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
