@@ -135,8 +135,9 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
 template <int D>
 struct BwdSmem {
   static constexpr int kBQ = (D == 128) ? 64 : 128;   // query rows per iteration
-  static constexpr int kNB = (D == 128) ? 2 : 1;      // S^T / dP^T / dS^T buffers (2 = pipelined)
-  static constexpr int kNQS = kNB + 1;                 // Q / dO / LSE2 / D stages
+  static constexpr int kNB = (D == 128) ? 2 : 1;      // S^T / dP^T TMEM buffers (2 = pipelined)
+  static constexpr int kNDS = 1;                       // dS^T staging buffers in shared memory
+  static constexpr int kNQS = (D == 128) ? 4 : 2;      // Q / dO / LSE2 / D stages
   static constexpr int kChunks = D / 64;
   static constexpr int kKVBytes = 128 * D * 2;         // one 128-key tile of K or V
   static constexpr int kQBytes = kBQ * D * 2;          // one query tile of Q or dO
@@ -146,7 +147,7 @@ struct BwdSmem {
   static constexpr int kQOff = kVOff + kKVBytes;
   static constexpr int kDOOff = kQOff + kNQS * kQBytes;
   static constexpr int kDSOff = kDOOff + kNQS * kQBytes;
-  static constexpr int kLOff = kDSOff + kNB * kDSBytes;   // LSE2 per stage, BQ floats
+  static constexpr int kLOff = kDSOff + kNDS * kDSBytes;  // LSE2 per stage, BQ floats
   static constexpr int kDVecOff = kLOff + kNQS * kBQ * 4;  // D_i per stage, BQ floats
   static constexpr int kBarOff = kDVecOff + kNQS * kBQ * 4;
   // kv_full, q_full[NQS], q_empty[NQS], sdp_full[NB], ds_ready[NB], dq_full[NB], dq_empty[NB], ds_empty[NB],
@@ -168,8 +169,9 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 // Pipeline (NB = 2): the MMA thread issues S^T/dP^T of tile it+2 right after dV/dK/dQ of tile it, so the
-// compute warps work on tile it+1 while the tensor core runs both. Buffers are indexed by it % NB, stages
-// of the Q/dO ring by it % NQS; every barrier's phases are waited in order.
+// compute warps work on tile it+1 while the tensor core runs both. TMEM buffers are indexed by it % NB, the
+// dS^T staging buffer by it % NDS, stages of the Q/dO ring by it % NQS (four stages for D = 128: a Q/dO tile
+// takes longer to arrive than two tiles take to process); every barrier's phases are waited in order.
 // kDrop: attention dropout; a separate instance so the plain path keeps its registers.
 template <int D, bool kBF16, bool kCausal, bool kDrop = false>
 __global__ void __launch_bounds__(384, 1)
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&ds_ready[x], (it / NB) & 1, abort_flag)) break;
         tc_fence_after_sync();
         const uint64_t qd = sdesc_add(q_mn, s * L::kQBytes), dod = sdesc_add(do_mn, s * L::kQBytes);
-        const uint64_t dsm = sdesc_add(ds_mn, x * L::kDSBytes);
+        const uint64_t dsm = sdesc_add(ds_mn, (it % L::kNDS) * L::kDSBytes);
         // dV += P^T dO and dK += dS^T Q, both with A from TMEM: the reduction runs over the BQ queries.
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk)
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_ss(tmem + L::kColS + x * BQ, a, bd, idesc_q, kk > 0);
         }
         umma_commit(&dq_full[x]);
-        umma_commit(&ds_empty[x]);
+        umma_commit(&ds_empty[it % L::kNDS]);
         umma_commit(&q_empty[s]);
         if (it + NB < n_it && !(issue_dp(it + NB) && issue_s(it + NB))) break;
       }
@@ -374,11 +376,12 @@ __global__ void __launch_bounds__(384, 1)
       const int x = it % NB, s = it % NQS;
       const int q0 = (i_begin + it % n_q) * BQ;
       if (!mbar_wait(&sdp_full[x], (it / NB) & 1, abort_flag)) { ok = false; break; }
-      if (it >= NB && !mbar_wait(&ds_empty[x], ((it / NB) - 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after_sync();
       const float* lse2 = reinterpret_cast<const float*>(smem + L::kLOff + s * BQ * 4);
       const float* dvec = reinterpret_cast<const float*>(smem + L::kDVecOff + s * BQ * 4);
-      uint8_t* ds_row_base = smem + L::kDSOff + x * L::kDSBytes + j * 128;
+      // dS^T staging buffer of this tile; the dQ product of the tile that used it before must have read it
+      // (waited for just before the first store, so the math overlaps that product).
+      uint8_t* ds_row_base = smem + L::kDSOff + (it % L::kNDS) * L::kDSBytes + j * 128;
       const uint32_t s_col = L::kColS + x * BQ, dp_col = L::kColDP + x * BQ;
       const int lo_c = has_right ? key - off - right - q0 : -1;
       const int hi_c = has_left ? key - off + p.win_left - q0 : BQ;
@@ -438,6 +441,9 @@ __global__ void __launch_bounds__(384, 1)
           // later, issued after the dK product, and the tensor core executes in issue order.
           tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
           // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
+          if (c0 == 0 && it >= L::kNDS &&
+              !mbar_wait(&ds_empty[it % L::kNDS], ((it / L::kNDS) - 1) & 1, abort_flag))
+            ok = false;
           uint8_t* row = ds_row_base + (c0 / 64) * 16384;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -479,6 +485,9 @@ __global__ void __launch_bounds__(384, 1)
           // later, issued after the dK product, and the tensor core executes in issue order.
           tmem_st_x32(lane_base + dp_col + c0 / 2, dk);
           // dS^T row j, queries c0..c0+63 = one whole 128-byte swizzled row of chunk c0/64.
+          if (c0 == 0 && it >= L::kNDS &&
+              !mbar_wait(&ds_empty[it % L::kNDS], ((it / L::kNDS) - 1) & 1, abort_flag))
+            ok = false;
           uint8_t* row = ds_row_base + (c0 / 64) * 16384;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -487,6 +496,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+      if (!ok) break;
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before_sync();
