@@ -31,9 +31,11 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 NOMINAL_BF16_TFLOPS = 2250.0
+_COMMON_SOURCES = ["exact_io_aware_76_b200/csrc/sm100.cuh", "exact_io_aware_76_b200/csrc/tmem_ldst.inc",
+                   "exact_io_aware_76_b200/csrc/dropout.cuh"]
 KERNEL_SOURCES = {
-    "fa_bwd_main": ["exact_io_aware_76_b200/csrc/fa_bwd.cuh", "exact_io_aware_76_b200/csrc/sm100.cuh"],
-    "fa_fwd": ["exact_io_aware_76_b200/csrc/fa_fwd.cuh", "exact_io_aware_76_b200/csrc/sm100.cuh"],
+    "fa_bwd_main": ["exact_io_aware_76_b200/csrc/fa_bwd.cuh"] + _COMMON_SOURCES,
+    "fa_fwd": ["exact_io_aware_76_b200/csrc/fa_fwd.cuh"] + _COMMON_SOURCES,
 }
 
 
