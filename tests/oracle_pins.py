@@ -25,7 +25,8 @@ What pins it:
     known-answer vectors and a keep block derived by hand from one of them (tests/golden/philox_dropout.json);
     dropout_p = 0 is the plain path; the keep rate matches 1 - t/256; O averaged over many seeds converges to
     the undropped O (the 1/(1 - p) rescale) with LSE unchanged; with V = I the output is P o Z itself; finite
-    differences with the mask held fixed.
+    differences with the mask held fixed;
+  * linearity in V: sum_j v_j . dV_j equals the loss sum_i dO_i . O_i, with and without dropout.
 """
 import json
 import math
@@ -515,9 +516,28 @@ def pin_dropout_finite_differences(orc):
             assert err <= 1e-6, ("dropout finite differences d" + name, err)
 
 
+def pin_value_linearity(orc):
+    # O is linear in V, so L = sum_i dO_i . O_i equals sum_j v_j . dV_j exactly (with or without dropout,
+    # grouped heads or a window): the gradient reaching V is the one that reproduces the loss.
+    r = _rng(20)
+    for (nq, nkv, Sq, Sk, D, causal, window, drop) in ((2, 2, 7, 9, 3, False, (-1, -1), None),
+                                                       (4, 2, 9, 9, 4, True, (3, 0), None),
+                                                       (2, 1, 8, 11, 3, False, (-1, -1), (0.3, 5, 2)),
+                                                       (2, 2, 10, 10, 2, True, (4, -1), (0.6, 9, 0))):
+        q = r.standard_normal((nq, Sq, D))
+        k = r.standard_normal((nkv, Sk, D))
+        v = r.standard_normal((nkv, Sk, D))
+        do = r.standard_normal((nq, Sq, D))
+        out, _ = orc.fwd(q, k, v, causal=causal, scale=0.6, window=window, dropout=drop)
+        _, _, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.6, window=window, dropout=drop)
+        loss = float(np.sum(out * do))
+        _close(float(np.sum(v * dv)), loss, tol=1e-10 * max(1.0, abs(loss)), what="sum v.dV = L")
+
+
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
             pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,
             pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_zero_is_plain, pin_dropout_keep_rate,
-            pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences]
+            pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences,
+            pin_value_linearity]
