@@ -430,10 +430,14 @@ __global__ void __launch_bounds__(384, 1)
           f2_unpack(sum2, s0, s1);
           sum = s0 + s1;
         };
-        if (need_mask)
-          p_loop(BoolTag<false>{});
-        else
-          p_loop(BoolTag<true>{});
+        if constexpr (L::kEmuEvery > 0) {
+          if (need_mask)
+            p_loop(BoolTag<false>{});
+          else
+            p_loop(BoolTag<true>{});
+        } else {
+          p_loop(BoolTag<false>{});  // one copy of the loop when both kinds of tile run the same code
+        }
       }
       l += sum;
       if (kFP8)
