@@ -394,9 +394,9 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       } else {
-        // p = 2^(s * scale_log2 - m) with packed pairs for the FMA and the row sum. In a tile without an
-        // element mask every x is finite, and every kEmuEvery-th group of four columns takes its exponentials
-        // from the FMA pipe (exp2_poly2), which relieves the MUFU unit that otherwise bounds this loop.
+        // p = 2^(s * scale_log2 - m) with packed pairs for the FMA and the row sum; with kEmuEvery > 0 every
+        // kEmuEvery-th group of four columns takes its exponentials from the FMA pipe (exp2_poly2), which
+        // relieves the MUFU unit (8-bit inputs only, where the tensor work per tile is half).
         auto p_loop = [&](auto emu_tag) {
           constexpr bool kEmu = decltype(emu_tag)::value && L::kEmuEvery > 0;
           const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m_use, -m_use);
@@ -430,14 +430,11 @@ __global__ void __launch_bounds__(384, 1)
           f2_unpack(sum2, s0, s1);
           sum = s0 + s1;
         };
-        if constexpr (L::kEmuEvery > 0) {
-          if (need_mask)
-            p_loop(BoolTag<false>{});
-          else
-            p_loop(BoolTag<true>{});
-        } else {
-          p_loop(BoolTag<false>{});  // one copy of the loop when both kinds of tile run the same code
-        }
+        // One copy of the loop for every tile (code size matters here: both softmax warpgroups stream it).
+        // With the FMA-pipe exponentials a masked element (x = -inf, clamped to -125) yields ~2^-125, which
+        // e4m3 rounds to exactly 0 for the PV product and which adds under 128 * 2^-125 to l; a row with no
+        // visible key keeps m = -inf, so its O (from P = 0) and LSE (-inf) are unchanged.
+        p_loop(BoolTag<(L::kEmuEvery > 0)>{});
       }
       l += sum;
       if (kFP8)
