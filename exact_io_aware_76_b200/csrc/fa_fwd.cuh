@@ -66,8 +66,8 @@ struct FwdSmem {
   static constexpr int kKOff = kQOff + kNQ * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 2 + 1;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], mma_done, p_half[2]
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 2 + 1 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B-swizzle atoms)
@@ -78,6 +78,9 @@ struct FwdSmem {
   // Measured on the GPT-shaped workload: with 8-bit inputs (half the MMA time per tile) one in four is
   // fastest (+5%); with 16-bit inputs any share made the kernel slower, so none.
   static constexpr int kEmuEvery = kFP8 ? 4 : 0;
+  // P is handed to the MMA thread in two halves of 64 keys (the first half of PV overlaps the second half of
+  // the exponentials). Measured: +4-6% with 8-bit inputs, -3% with 16-bit ones (one hand-off is cheaper there).
+  static constexpr bool kSplitP = kFP8;
 };
 
 // kBF16: the 16-bit input type (and output type); with kFP8 the inputs are e4m3 and the output is bf16.
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* mma_done = o_full + 2;
+  uint64_t* p_half = mma_done + 1;  // P of keys 0..63 is in TMEM (the first half of PV may start)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -158,6 +162,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
+      mbar_init(&p_half[t], 128);
       mbar_init(&o_full[t], 1);
     }
     mbar_init(mma_done, 1);
@@ -245,13 +250,15 @@ __global__ void __launch_bounds__(384, 1)
       };
       // O_t += P_t V_j : A = P_t from TMEM (8 columns per instruction: 16 keys of 16-bit P, or 32 keys of e4m3
       // P), B = V_j MN-major (as many 128-byte key rows per instruction; 64-wide head-dim blocks 16 KB apart).
-      auto issue_pv = [&](int t, int s, bool acc) {
+      // Issued in two halves of 64 keys (with kSplitP the softmax publishes P of keys 0..63 first).
+      auto issue_pv = [&](int t, int s, bool acc, int half) {
         const uint32_t o_tmem = tmem + 256 + t * D;
         const uint32_t p_tmem = tmem + t * 128;
         const uint64_t b0 = sdesc_add(v_desc, s * L::kTileBytes);
         constexpr int kKeys = kFP8 ? 32 : 16;  // keys per instruction
+        constexpr int kHalf = 64 / kKeys;      // instructions per half
 #pragma unroll
-        for (int kk = 0; kk < 128 / kKeys; ++kk) {
+        for (int kk = half * kHalf; kk < (half + 1) * kHalf; ++kk) {
           if (kFP8)
             umma_ts_f8(o_tmem, p_tmem + kk * 8, sdesc_add(b0, kk * kKeys * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
           else
@@ -277,9 +284,14 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2 && ok; ++t) {
           if (n_kv[t] == 0 || jj < j_lo[t] || jj >= j_lo[t] + n_kv[t]) continue;
           const int u = jj - j_lo[t];  // this tile's local step
-          if (!mbar_wait(&p_full[t], u & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(L::kSplitP ? &p_half[t] : &p_full[t], u & 1, abort_flag)) { ok = false; break; }
           tc_fence_after_sync();
-          issue_pv(t, s, u > 0);
+          issue_pv(t, s, u > 0, 0);
+          if (L::kSplitP) {
+            if (!mbar_wait(&p_full[t], u & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after_sync();
+          }
+          issue_pv(t, s, true, 1);
           umma_commit(&o_full[t]);
           if (u + 1 < n_kv[t]) {
             if (!next_k_ready) {
@@ -367,6 +379,27 @@ __global__ void __launch_bounds__(384, 1)
       const float m_use = (m == -INFINITY) ? 0.f : m;
       float sum = 0.f;
       uint32_t pk[L::kPCols];
+      // With kSplitP: P of keys 64*half .. 64*half+63 -> TMEM, then p_half (half 0) or p_full (half 1), so the
+      // MMA thread starts the first half of PV while this thread computes the second half of the row.
+      // Without it: all of P -> TMEM, then p_full, once.
+      auto publish = [&](auto half_tag) {
+        constexpr int half = decltype(half_tag)::value ? 1 : 0;
+        if constexpr (L::kSplitP) {
+          if constexpr (kFP8)
+            tmem_st_x16(s_tmem + half * 16, pk + half * 16);
+          else
+            tmem_st_x32(s_tmem + half * 32, pk + half * 32);
+        } else {
+          if constexpr (half == 0) return;
+          if constexpr (kFP8)
+            tmem_st_x32(s_tmem, pk);
+          else
+            tmem_st_x64(s_tmem, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        mbar_arrive(half ? &p_full[t] : &p_half[t]);
+      };
       if constexpr (kDrop && !kFP8) {
         // Dropout: P keeps only the kept probabilities (l sums them all; 1/(1-t/256) is applied to O at the
         // end). Per 16 keys, the four lanes of this row's 4-row block each generate one 4x4 block of the mask
@@ -392,6 +425,7 @@ __global__ void __launch_bounds__(384, 1)
             pk[c / 2] = pack2<kBF16>(p0, p1);
             pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
           }
+          if (c16 == 48) publish(BoolTag<false>{});
         }
       } else {
         // p = 2^(s * scale_log2 - m) with packed pairs for the FMA and the row sum; with kEmuEvery > 0 every
@@ -425,6 +459,7 @@ __global__ void __launch_bounds__(384, 1)
               pk[c / 2] = pack2<kBF16>(p0, p1);
               pk[c / 2 + 1] = pack2<kBF16>(p2, p3);
             }
+            if (c == 60) publish(BoolTag<false>{});
           }
           float s0, s1;
           f2_unpack(sum2, s0, s1);
@@ -437,13 +472,7 @@ __global__ void __launch_bounds__(384, 1)
         p_loop(BoolTag<(L::kEmuEvery > 0)>{});
       }
       l += sum;
-      if (kFP8)
-        tmem_st_x32(s_tmem, pk);
-      else
-        tmem_st_x64(s_tmem, pk);
-      tmem_st_wait();
-      tc_fence_before_sync();
-      mbar_arrive(&p_full[t]);
+      publish(BoolTag<true>{});
     }
     // ---------------------------------------------------------------- epilogue: O / l and LSE
     if (ok && nt > 0) ok = mbar_wait(&o_full[t], (nt - 1) & 1, abort_flag);
