@@ -479,7 +479,9 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after_sync();
       const bool valid_row = row < p.Sq;
-      const float inv_l = (l > 0.f) ? p.v_descale / l : 0.f;
+      // A row that never saw a visible key (m = -inf) has O = 0: its l may hold the ~2^-125 weights that the
+      // FMA-pipe exponentials give masked elements.
+      const float inv_l = (l > 0.f && m != -INFINITY) ? p.v_descale / l : 0.f;
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + ((static_cast<size_t>(b) * p.Sq + row) * p.H + h) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
