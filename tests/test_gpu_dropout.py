@@ -16,6 +16,7 @@ import torch
 import exact_io_aware_76_b200 as fa
 import oracle
 from exact_io_aware_76_b200.inputs import draw
+from exact_io_aware_76_b200.workloads import WORKLOADS, make_workload_inputs
 from parity_util import (all_heads, check_grad, check_lse, check_out, gather_lse, gather_rows, heads_f64, kv_heads)
 
 pytestmark = pytest.mark.gpu
@@ -122,3 +123,38 @@ def test_zero_probability_is_the_plain_kernel():
     assert rc == 0
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_gpt_workload_sampled_rows():
+    """The GPT-shaped workload (4x32x8192x128 bf16 causal) with dropout 0.1: O and LSE on 4 sampled rows of every
+    head; dQ of those rows and their dK/dV contributions (a second backward with dO zeroed on every other row,
+    which removes exactly the other rows' terms)."""
+    w = WORKLOADS["gpt"]
+    q, k, v, do = make_workload_inputs(w, with_dout=True)
+    p, seed, offset = 0.1, 20240601, 17
+    kw = dict(causal=True, dropout_p=p, seed=seed, offset=offset)
+    out, lse = fa.fwd(q, k, v, **kw)
+    heads = all_heads(w.B, w.H)
+    r = np.random.default_rng(5)
+    rows = np.stack([np.array([0, w.Sq - 1, 127, 128], np.int64) if t % 2 == 0
+                     else np.sort(r.choice(w.Sq, 4, replace=False)).astype(np.int64) for t in range(len(heads))])
+    mask = torch.zeros(w.B, w.Sq, w.H, 1, dtype=do.dtype, device=do.device)
+    for t, (b, h) in enumerate(heads):
+        mask[b, torch.as_tensor(rows[t], device=do.device), h] = 1
+    dq, _, _ = fa.bwd(q, k, v, out, lse, do, **kw)
+    _, dk_m, dv_m = fa.bwd(q, k, v, out, lse, do * mask, **kw)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    for c0 in range(0, len(heads), 16):
+        sub = heads[c0:c0 + 16]
+        sr = rows[c0:c0 + 16]
+        hi = head_numbers(sub, w.H)
+        args = (heads_f64(q, sub), heads_f64(k, sub), heads_f64(v, sub))
+        o_ref, l_ref = oracle.attn_fwd(*args, causal=True, rows=sr, dropout=(p, seed, offset), head_index=hi)
+        check_out(gather_rows(out, sub, sr), o_ref, q.dtype, sigma=rescale(p))
+        check_lse(gather_lse(lse, sub, sr), l_ref)
+        dq_r, dk_r, dv_r = oracle.attn_bwd(*args, heads_f64(do, sub), causal=True, rows=sr,
+                                           dropout=(p, seed, offset), head_index=hi)
+        check_grad(gather_rows(dq, sub, sr), dq_r, "dQ sampled rows")
+        check_grad(gather_rows(dk_m, sub), dk_r, "dK of sampled rows")
+        check_grad(gather_rows(dv_m, sub), dv_r, "dV of sampled rows")

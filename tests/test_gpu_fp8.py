@@ -25,7 +25,8 @@ import torch
 import exact_io_aware_76_b200 as fa
 import oracle
 from exact_io_aware_76_b200.inputs import draw_e4m3
-from parity_util import check_lse, gather_lse, gather_rows, half_ulp
+from exact_io_aware_76_b200.workloads import WORKLOADS, make_workload_inputs
+from parity_util import all_heads, check_lse, gather_lse, gather_rows, half_ulp
 
 pytestmark = pytest.mark.gpu
 
@@ -34,14 +35,14 @@ def deq(x, d, b, h):
     return x[b, :, h, :].to("cpu", torch.float64).numpy() * d
 
 
-def visible_mask(Sq, Sk, causal, window):
-    i = np.arange(Sq)[:, None]
+def visible_mask(Sq, Sk, causal, window, rows=None):
+    i = (np.arange(Sq) if rows is None else np.asarray(rows))[:, None]
     j = np.arange(Sk)[None, :]
     c = i + (Sk - Sq)
     left, right = window
     if causal:
         right = 0 if right < 0 else min(right, 0)
-    vis = np.ones((Sq, Sk), bool)
+    vis = np.ones((i.shape[0], Sk), bool)
     if left >= 0:
         vis &= j >= c - left
     if right >= 0:
@@ -54,11 +55,12 @@ def oracle_heads(qs, ks, vs, causal, scale, window):
     return o, l
 
 
-def bound(qh, kh, vh, causal, scale, window):
-    """Per-element bound on |O - O_ref| from rounding the probabilities to e4m3 (see the module docstring)."""
+def bound(qh, kh, vh, causal, scale, window, rows=None):
+    """Per-element bound on |O - O_ref| from rounding the probabilities to e4m3 (see the module docstring), for
+    every row of qh or only the listed rows."""
     Sq, Sk = qh.shape[0], kh.shape[0]
-    vis = visible_mask(Sq, Sk, causal, window)
-    s = scale * (qh @ kh.T)
+    vis = visible_mask(Sq, Sk, causal, window, rows)
+    s = scale * ((qh if rows is None else qh[rows]) @ kh.T)
     s = np.where(vis, s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     has = np.isfinite(m)
@@ -142,3 +144,32 @@ def test_fp8_forward_exact_when_probabilities_are_powers_of_two(causal, window, 
     bd = half_ulp(o_ref, torch.bfloat16) + 1e-4 * vmax
     assert np.all(err <= bd), "max err %.3e, max err/bound %.3f" % (float(err.max()), float((err / bd).max()))
     print(check_lse(gather_lse(lse, heads), l_ref))
+
+
+@pytest.mark.parametrize("name,n_heads,per_head", [("gpt", 128, 4), ("long", 8, 4)])
+def test_fp8_full_size_sampled_rows(name, n_heads, per_head):
+    """The GPT-shaped (4x32x8192x128) and long-context (1x32x131072x128) workloads in e4m3, on sampled rows
+    (first, last, both sides of the first tile edge and random) of n_heads evenly spaced heads."""
+    w = WORKLOADS[name]
+    q, k, v = make_workload_inputs(w)
+    q8, k8, v8 = (x.to(torch.float8_e4m3fn) for x in (q, k, v))
+    del q, k, v
+    out, lse = fa.fwd_fp8(q8, k8, v8, causal=w.causal)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    heads = all_heads(w.B, w.H)
+    heads = heads[::max(1, len(heads) // n_heads)][:n_heads]
+    r = np.random.default_rng(11)
+    scale = 1.0 / math.sqrt(w.D)
+    worst = 0.0
+    for (b, h) in heads:
+        rows = np.array([0, w.Sq - 1, 127, 128] + list(r.choice(w.Sq, per_head, replace=False)), np.int64)
+        qh, kh, vh = deq(q8, 1.0, b, h), deq(k8, 1.0, b, h), deq(v8, 1.0, b, h)
+        o_ref, l_ref = oracle.attn_fwd(qh[None], kh[None], vh[None], causal=w.causal, scale=scale, rows=rows[None])
+        bd = bound(qh, kh, vh, w.causal, scale, (-1, -1), rows) + half_ulp(o_ref[0], torch.bfloat16)
+        o = gather_rows(out, [(b, h)], [rows])[0]
+        err = np.abs(o - o_ref[0])
+        worst = max(worst, float((err / bd).max()))
+        assert np.all(err <= bd), "head (%d,%d): max err/bound %.3f" % (b, h, float((err / bd).max()))
+        check_lse(gather_lse(lse, [(b, h)], [rows]), l_ref)
+    print("max err/bound %.3f over %d heads" % (worst, len(heads)))
