@@ -1,6 +1,7 @@
 """Build the CUDA libraries in-tree with nvcc for sm_100a.
 
-  libfa.so           the product: fa_fwd / fa_bwd / fa_bwd_workspace_size / fa_status_string / fa_device_status
+  libfa.so           the product: the entry points of include/fa.h (fa_fwd, fa_bwd and their _ex, _fp8,
+                     _dropout, _noalloc and _stage forms, fa_bwd_workspace_size, fa_status_string, fa_device_status)
   libfa_selftest.so  test-only one-CTA tcgen05 products that check the layout conventions the kernels use
 
 Run ``python -m exact_io_aware_76_b200.build`` (or ``__graft_entry__.build()``).
