@@ -63,43 +63,72 @@ constexpr float kLog2eB = 1.4426950408889634f;
 // One warp per (b, s, h) row: D = sum_d dO*O in fp32. Then zero dQacc with 16-byte stores.
 template <int D, bool kBF16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
+  // A row of O / dO is D 16-bit values = D / 8 lanes x 16 bytes, so one 16-byte load instruction of a warp
+  // covers 256 / D rows; two of them per iteration keep four independent loads in flight per lane.
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerLoad = 32 / kLanesPerRow;
+  constexpr int kUnroll = 2;
+  constexpr int kRowsPerIter = kRowsPerLoad * kUnroll;
   const int warps_total = gridDim.x * 8;
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow;    // which row of the load this lane works on
+  const int part = lane % kLanesPerRow;   // which 16-byte piece of that row
   const long long rows = (long long)p.B * p.H * p.Sq_pad;
-  constexpr int kPer = D / 32;  // elements per lane
-  for (long long r = gw; r < rows; r += warps_total) {
-    const int i = (int)(r % p.Sq_pad);
-    const long long bh = r / p.Sq_pad;
-    const int b = (int)(bh / p.H), h = (int)(bh % p.H);
-    float acc = 0.f;
-    if (i < p.Sq) {
-      const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.H + h) * D + lane * kPer;
-      const uint16_t* o = reinterpret_cast<const uint16_t*>(p.out) + base;
-      const uint16_t* g = reinterpret_cast<const uint16_t*>(p.dout) + base;
+  for (long long r0 = (long long)gw * kRowsPerIter; r0 < rows; r0 += (long long)warps_total * kRowsPerIter) {
+    uint4 ov[kUnroll], gv[kUnroll];
+    long long rr[kUnroll];
+    bool live[kUnroll];
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) {
-        float a, c;
-        if (kBF16) {
-          a = __uint_as_float(static_cast<uint32_t>(o[e]) << 16);
-          c = __uint_as_float(static_cast<uint32_t>(g[e]) << 16);
-        } else {
-          a = __half2float(__ushort_as_half(o[e]));
-          c = __half2float(__ushort_as_half(g[e]));
-        }
-        acc = fmaf(a, c, acc);
+    for (int u = 0; u < kUnroll; ++u) {
+      rr[u] = r0 + u * kRowsPerLoad + sub;
+      const int i = (int)(rr[u] % p.Sq_pad);
+      const long long bh = rr[u] / p.Sq_pad;
+      live[u] = rr[u] < rows && i < p.Sq;
+      ov[u] = gv[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (live[u]) {
+        const int b = (int)(bh / p.H), h = (int)(bh % p.H);
+        const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.H + h) * D + part * 8;
+        ov[u] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.out) + base);
+        gv[u] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + base);
       }
     }
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (lane == 0) {
-      float l2 = INFINITY;  // padding rows and rows that see no key: P = 2^(s - inf) = 0
-      if (i < p.Sq) {
-        const float l = p.lse[(static_cast<size_t>(b) * p.H + h) * p.Sq + i];
-        if (l != -INFINITY) l2 = l * kLog2eB;
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t* o32 = reinterpret_cast<const uint32_t*>(&ov[u]);
+      const uint32_t* g32 = reinterpret_cast<const uint32_t*>(&gv[u]);
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a0, a1, c0, c1;
+        if (kBF16) {
+          a0 = __uint_as_float(o32[e] << 16);
+          a1 = __uint_as_float(o32[e] & 0xffff0000u);
+          c0 = __uint_as_float(g32[e] << 16);
+          c1 = __uint_as_float(g32[e] & 0xffff0000u);
+        } else {
+          a0 = __half2float(__ushort_as_half(static_cast<uint16_t>(o32[e] & 0xffffu)));
+          a1 = __half2float(__ushort_as_half(static_cast<uint16_t>(o32[e] >> 16)));
+          c0 = __half2float(__ushort_as_half(static_cast<uint16_t>(g32[e] & 0xffffu)));
+          c1 = __half2float(__ushort_as_half(static_cast<uint16_t>(g32[e] >> 16)));
+        }
+        acc = fmaf(a1, c1, fmaf(a0, c0, acc));
       }
-      p.dvec[r] = (i < p.Sq) ? acc : 0.f;
-      p.lse2[r] = l2;
+      // reduce over the lanes of this row (aligned groups of kLanesPerRow lanes)
+#pragma unroll
+      for (int s = kLanesPerRow / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+      if (part == 0 && rr[u] < rows) {
+        const long long r = rr[u];
+        const int i = (int)(r % p.Sq_pad);
+        const long long bh = r / p.Sq_pad;
+        float l2 = INFINITY;  // padding rows and rows that see no key: P = 2^(s - inf) = 0
+        if (i < p.Sq) {
+          const float l = p.lse[bh * p.Sq + i];
+          if (l != -INFINITY) l2 = l * kLog2eB;
+        }
+        p.dvec[r] = (i < p.Sq) ? acc : 0.f;
+        p.lse2[r] = l2;
+      }
     }
   }
   const long long n4 = (long long)p.B * p.H * p.Sq_pad * D / 4;
