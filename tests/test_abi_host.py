@@ -112,3 +112,11 @@ def test_dropout_rejects_bad_probability(p):
 def test_dropout_rejects_bad_shapes_first():
     assert fwd_drop_call(0.1, B=0) == -1
     assert fwd_drop_call(0.1, D=96) == -2
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    # No fallback: without the built library the binding raises instead of computing anything elsewhere.
+    monkeypatch.setattr(fa, "_lib", None)
+    monkeypatch.setattr(fa, "LIB_PATH", str(tmp_path / "libfa.so"))
+    with pytest.raises(ImportError):
+        fa.lib()
