@@ -1,5 +1,5 @@
 // fa_api.cu -- the C ABI of libfa.so (declared in include/fa.h): argument validation, TMA descriptor
-// encoding, kernel selection by (head dim, dtype, causal) and launch on the caller's stream.
+// encoding, kernel selection by (head dim, dtype, causal, e4m3, dropout) and launch on the caller's stream.
 #include <cudaTypedefs.h>
 #include <math.h>
 

@@ -11,7 +11,7 @@
 // Three kernels, in stream order:
 //   fa_bwd_pre   D_i and LSE_i*log2(e) into the workspace (padded to a 128-row multiple), zero the fp32 dQ
 //                accumulator. HBM-bound elementwise work.
-//   fa_bwd_main  one CTA per (batch, head, 128-key tile); loops over the query tiles that see those keys.
+//   fa_bwd_main  one CTA per (batch, K/V head, 128-key tile); loops over the query tiles that see its keys.
 //   fa_bwd_dq    dQ = dtype(scale * dQacc), HBM-bound.
 //
 // fa_bwd_main warp roles:
@@ -22,8 +22,8 @@
 //              (times scale) and dV.
 //   warps 4-7  "dQ": read each dQ partial out of TMEM and add it to the fp32 accumulator in L2 with coalesced
 //              reductions straight from registers.
-//   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 3-stage (D=128) or 2-stage
-//              ring.
+//   warp 8     TMA producer: K, V once; Q, dO, LSE2, D per query tile through a 4-stage (D=128) or 2-stage
+//              ring (every query head of the K/V head's group in turn).
 //   warp 9     TMEM allocator and tcgen05 MMA issuer.
 // Per query tile the MMAs are: dP^T = V dO^T, S^T = K Q^T (into TMEM), then dV += P^T dO and dK += dS^T Q
 // (A from TMEM), and dQ^T = K^T dS^T (D = 128; lane = head-dim index) or dQ = dS K (D = 64; lane = query),

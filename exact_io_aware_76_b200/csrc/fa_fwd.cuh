@@ -16,8 +16,8 @@
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go to the softmax warpgroups)
 // Registers: 384 threads x 168 at launch; setmaxnreg moves the third warpgroup to 88 and the two softmax
 // warpgroups to 208 (2*128*208 + 128*88 = 64512 = 384*168), enough to hold a full 128-column S row.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D). P_t (16-bit) overwrites the
-// first 64 columns of S_t and is the A operand of the PV MMA read straight from TMEM.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D). P_t overwrites the first 64
+// (16-bit P) or 32 (e4m3 P) columns of S_t and is the A operand of the PV MMA read straight from TMEM.
 // The MMA issue order is S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ..., so while one warpgroup runs the
 // softmax of its tile the tensor core works on the other tile (ping-pong).
 //

@@ -125,47 +125,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// Bulk reduction shared -> global: dst[i] += src[i] for `bytes`/4 floats, performed at L2 by the copy engine
-// (dst, src and bytes multiples of 16). Completion is tracked per issuing thread with bulk groups.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until this thread's committed bulk groups have finished reading their shared-memory sources.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Wait until this thread's committed bulk groups have completed entirely.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Named barrier over `count` threads (a multiple of 32; whole warps).
-template <int kId, int kCount>
-__device__ __forceinline__ void named_bar_sync() {
-  asm volatile("bar.sync %0, %1;" ::"n"(kId), "n"(kCount) : "memory");
-}
-// Named barrier that also returns the AND of `pred` over the participating threads, so that a group can take
-// a uniform decision (e.g. every thread leaves a loop together after one of them gave up on a wait).
-template <int kId, int kCount>
-__device__ __forceinline__ bool named_bar_and(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "n"(kId), "n"(kCount)
-      : "memory");
-  return r != 0;
-}
-
 // ---------------------------------------------------------------------------------------------------------
-// tcgen05: tensor memory and the 5th-generation tensor-core MMA
+// tcgen05: tensor memory and the 5th-generation tensor-core MMA. A TMEM address holds the lane in bits 31..16
+// and the (32-bit) column in bits 15..0.
 // ---------------------------------------------------------------------------------------------------------
-// TMEM address: bits 31..16 lane, bits 15..0 column (32-bit columns).
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
-  return base + (lane << 16) + col;
-}
-
 // Whole warp: allocate `ncols` columns (power of two >= 32); the address is written to *smem_dst.
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_dst)),

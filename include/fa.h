@@ -15,8 +15,10 @@
  * Conventions shared by every entry point
  *   - Layout [batch, seqlen, nheads, headdim] ("[batch, seqlen, nheads, headdim]" in the skill page's
  *     flash_attn_func examples), contiguous, row-major: element (b, s, h, d) sits at ((b*S + s)*H + h)*D + d.
- *     q, out, dout, dq: [B, Sq, H, D];  k, v, dk, dv: [B, Sk, H, D];  lse: fp32 [B, H, Sq].
- *   - dtype: FA_F16 or FA_BF16 for every 16-bit tensor of a call (the pages: fp16/bf16 only, no fp32).
+ *     q, out, dout, dq: [B, Sq, H, D];  k, v, dk, dv: [B, Sk, H, D] ([B, Sk, Hkv, D] in the entry points
+ *     that take Hkv);  lse: fp32 [B, H, Sq].
+ *   - dtype: FA_F16 or FA_BF16 for every 16-bit tensor of a call (the pages: fp16/bf16 only, no fp32); the
+ *     e4m3 forward (fa_fwd_fp8) takes 8-bit q, k, v and writes bf16.
  *   - D (head dim) in {64, 128}. B, H, Sq, Sk >= 1. Every pointer 16-byte aligned, device memory.
  *   - scale: 0.0f means 1/sqrt(D) (the pages' softmax_scale=None "Auto-scale"); any other finite value is
  *     used as given.
