@@ -11,9 +11,8 @@ bf16, causal, with q, k, v and dO iid N(0,1) from a fixed seed. FLOPs: forward 4
 Prints one JSON line (rank 0). ``value`` is the whole-job TFLOP/s from CUDA events with the inputs resident
 in HBM (1.07 GB per step, larger than the 126 MB L2); ``e2e`` is the same metric through the public Python API
 with pinned host inputs copied in and the gradients copied out every step (two buffer sets on separate upload,
-compute and download streams, so step i+1's upload and step i-1's download overlap step i); ``roofline`` rates
-the dominant
-kernel against the measured bf16 peak; ``cpu_baseline`` times the fp64 CPU oracle on a bounded row sample.
+compute and download streams, so step i+1's upload and step i-1's download overlap step i); ``roofline``
+rates the dominant kernel against the measured bf16 peak; ``cpu_baseline`` times the fp64 CPU oracle on a bounded row sample.
 With N > 1 (torchrun) every GPU runs its own replica of the workload (weak scaling, no collective on the data
 path) and the time is the maximum over ranks. ``--impl reference`` times the oracle itself as the reference
 arm (rank 0 only).
