@@ -26,6 +26,8 @@ def test_usage_example():
     for t in (out, lse, dq, dk, dv, out_g, out_d, lse_d, out8, lse8):
         assert torch.isfinite(t.float()).all()
     assert torch.equal(out_d0, out) and torch.equal(lse_d0, lse)   # dropout_p = 0 is the plain forward
-    assert torch.equal(lse_d, lse)                                  # dropout leaves the LSE unchanged
+    # dropout leaves the LSE unchanged (up to the order of the fp32 row sum, which the dropout loop forms in
+    # groups of 16 keys)
+    assert (lse_d - lse).abs().max() <= 1e-5
     assert (out_d.float() - out.float()).abs().max() > 0            # but not the output
     assert (lse8 - lse).abs().max() < 0.5                           # e4m3 inputs: the same scores, rounded
