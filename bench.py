@@ -200,6 +200,25 @@ def oracle_sample(w, q, k, v, do, seconds, seed=0):
     return fl / dt / 1e12, desc, threads, dt
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_record(w, value, threads, desc):
+    """The oracle's sampled rate, the host it ran on, and the time the whole problem would take at that rate
+    (an extrapolation, labelled as one)."""
+    full = w.fwd_flops() + (0 if w.name.startswith("long") else w.bwd_flops())
+    return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+            "cpu_model": cpu_model(), "extrapolated_full_problem_s": full / (value * 1e12) if value > 0 else None}
+
+
 # ------------------------------------------------------------------------------------------------ arms
 def run_reference(args):
     from exact_io_aware_76_b200.inputs import make_inputs
@@ -225,7 +244,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": workload_config(w, 1),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "cpu_baseline": cpu_baseline_record(w, value, threads, desc),
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -302,6 +321,9 @@ def run_ours(args):
     t_host1 = time.time()
     replicas.barrier(dev)
     local_ms = start.elapsed_time(stop)
+    # O(N) memory: everything the step holds on the device (inputs, outputs, workspace) against what one S x S
+    # bf16 score matrix per (batch, head) would take.
+    peak_bytes = torch.cuda.max_memory_allocated(dev)
     max_ms = replicas.max_over_ranks(local_ms, dev)
     if rank == 0:
         sampler.stop()
@@ -404,7 +426,7 @@ def run_ours(args):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         val, desc, threads, _ = oracle_sample(w, q, k, v, do, args.cpu_seconds)
-        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline_record(w, val, threads, desc)
     clocks = sampler.summary(t_host0, t_host1)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -412,7 +434,12 @@ def run_ours(args):
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(names) * K, "clocks": clocks,
             "fwd_tflops": kernels["fa_fwd"]["tflops"],
             "fwd_frac_of_measured_peak": kernels["fa_fwd"]["tflops"] / peaks["bf16_tflops"],
-            "kernels": kernels}
+            "kernels": kernels,
+            # model FLOPs: the backward without its recomputed Q K^T (8*B*H*D*pairs), alongside the
+            # algorithmic 10*B*H*D*pairs that `value` uses
+            "step_model_tflops": (flops_fwd + 0.8 * flops_bwd) * world * K / (max_ms / 1e3) / 1e12,
+            "memory": {"peak_device_bytes": peak_bytes,
+                       "score_matrix_bf16_bytes": 2 * w.B * w.H * w.Sq * w.Sk}}
     if not fwd_only:
         line["bwd_tflops"] = flops_bwd / (bwd_ms / 1e3) / 1e12
         line["bwd_frac_of_measured_peak"] = line["bwd_tflops"] / peaks["bf16_tflops"]

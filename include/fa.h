@@ -26,7 +26,8 @@
  *     iff j <= i + (Sk - Sq). A query row that sees no key gets O = 0 and LSE = -inf.
  *   - lse[b,h,i] = ln sum_{j visible} exp(scale * q_i . k_j), fp32 (natural log, scale included).
  *   - Ownership: the caller allocates and owns every buffer, including the backward workspace. The library
- *     allocates no device memory; it keeps no per-call state besides a device-side sticky error word.
+ *     allocates no device memory; it keeps no per-call state besides a device-side sticky error word and a
+ *     small host-side cache of encoded TMA descriptors (keyed by pointer and shape, so reusing a buffer is safe).
  *   - Asynchrony: all work is enqueued on `stream` (0 = legacy default stream). A return of FA_OK means the
  *     launches were accepted, not that they finished. A kernel that gives up on an internal wait (bounded
  *     spin, about 2 s) records FA_ERR_TIMEOUT in the device status word (fa_device_status) and exits cleanly.
