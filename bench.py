@@ -253,14 +253,23 @@ def run_reference(args):
 METRIC = "attention fwd/bwd TFLOP/s (bf16, causal) and % of B200 dense tensor peak"
 
 
+L2_BYTES = 126 << 20
+
+
+def input_bytes(w):
+    """Bytes one step reads as its inputs (q, k, v, and dO for a training step)."""
+    return (3 if w.name.startswith("long") else 4) * w.B * w.Sq * w.H * w.D * 2
+
+
 def workload_config(w, n):
     kind = "forward" if w.name.startswith("long") else "training step (forward + recomputation backward)"
     return {"workload": "%s %s: B=%d H=%d Sq=%d Sk=%d D=%d %s %s" % (
                 w.name, kind, w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, "causal" if w.causal else "non-causal"),
             "global_batch": w.B * n, "seq_len": w.Sq,
             "parallelism": "replicas x%d (weak scaling; no collective on the data path)" % n,
-            "l2": "inputs larger than L2 (%.2f GB per step)" % (
-                (3 if w.name.startswith("long") else 4) * w.B * w.Sq * w.H * w.D * 2 / 1e9)}
+            "l2": ("inputs larger than L2 (%.2f GB per step)" % (input_bytes(w) / 1e9)) if input_bytes(w) >= L2_BYTES
+            else ("L2 flushed before every timed step by a 256 MB write outside the step's events (inputs %.3f GB)"
+                  % (input_bytes(w) / 1e9))}
 
 
 def run_ours(args):
@@ -304,6 +313,10 @@ def run_ours(args):
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    # Inputs that fit in L2 would be re-read from it by the next step: then a 256 MB write (twice the 126 MB
+    # L2) runs before every timed step, outside the step's own events, and `value` comes from those events.
+    flush_l2 = input_bytes(w) < L2_BYTES
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(str(getattr(props, "uuid", "")))
     if rank == 0:
@@ -315,12 +328,16 @@ def run_ours(args):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(K):
+        if flush_l2:
+            flush_buf.zero_()
         step(evs[i])
     stop.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.time()
     replicas.barrier(dev)
     local_ms = start.elapsed_time(stop)
+    if flush_l2:
+        local_ms = sum(evs[i][0].elapsed_time(evs[i][-1]) for i in range(K))
     # O(N) memory: everything the step holds on the device (inputs, outputs, workspace) against what one S x S
     # bf16 score matrix per (batch, head) would take.
     peak_bytes = torch.cuda.max_memory_allocated(dev)
