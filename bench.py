@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller cases for profiling)")
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller cases for profiling)")
+    ap.add_argument("--variant", choices=["plain", "fp8", "dropout"], default="plain",
+                    help="fp8: the e4m3 forward alone; dropout: forward + backward with dropout_p 0.1")
     return ap.parse_args()
 
 
@@ -261,6 +263,17 @@ def input_bytes(w):
     return (3 if w.name.startswith("long") else 4) * w.B * w.Sq * w.H * w.D * 2
 
 
+def variant_config(cfg, variant):
+    """The workload description of a --variant run (the plain run keeps the workload's own)."""
+    cfg = dict(cfg, variant=variant)
+    if variant == "fp8":
+        cfg["workload"] = cfg["workload"].replace("training step (forward + recomputation backward)",
+                                                  "forward on e4m3 inputs (descale 1), bf16 output")
+    elif variant == "dropout":
+        cfg["workload"] += ", attention dropout_p 0.1 (Philox seed 1234, offset 0)"
+    return cfg
+
+
 def workload_config(w, n):
     kind = "forward" if w.name.startswith("long") else "training step (forward + recomputation backward)"
     return {"workload": "%s %s: B=%d H=%d Sq=%d Sk=%d D=%d %s %s" % (
@@ -284,27 +297,48 @@ def run_ours(args):
     dev = torch.device("cuda", local_rank)
     replicas.init("nccl" if world > 1 else "gloo")
     w = workload_from_args(args)
-    fwd_only = w.name.startswith("long")
+    variant = args.variant
+    fwd_only = w.name.startswith("long") or variant == "fp8"
     seed = replicas.replica_seed(w.seed, rank)
     q, k, v, do = make_inputs(w.B, w.Sq, w.Sk, w.H, w.D, w.dtype, seed, w.sigma, "cuda", with_dout=True)
     out = torch.empty_like(q)
+    if variant == "fp8":  # the same draws rounded to e4m3 (descale 1); the output stays bf16
+        q, k, v = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    drop = dict(dropout_p=0.1, seed=1234, offset=0) if variant == "dropout" else {}
+
+    def fwd_call(q_, k_, v_, out_, lse_):
+        if variant == "fp8":
+            return fa.fwd_fp8(q_, k_, v_, causal=w.causal, out=out_, lse=lse_)
+        return fa.fwd(q_, k_, v_, causal=w.causal, out=out_, lse=lse_, **drop)
+
     lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.workspace_size(w.B, w.Sq, w.H, w.D), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    names = ["fa_fwd"] if fwd_only else ["fa_fwd", "fa_bwd_pre", "fa_bwd_main", "fa_bwd_dq"]
+    if fwd_only:
+        names = ["fa_fwd"]
+    elif variant == "dropout":  # the backward's launches are not separable with dropout: timed as one interval
+        names = ["fa_fwd", "fa_bwd"]
+    else:
+        names = ["fa_fwd", "fa_bwd_pre", "fa_bwd_main", "fa_bwd_dq"]
 
     def step(evs=None):
         def mark(i):
             if evs is not None:
                 evs[i].record(stream)
         mark(0)
-        fa.fwd(q, k, v, causal=w.causal, out=out, lse=lse)
+        fwd_call(q, k, v, out, lse)
         mark(1)
-        if not fwd_only:
-            for st in range(3):
-                fa.bwd(q, k, v, out, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, stage=st)
-                mark(2 + st)
+        if fwd_only:
+            return
+        if variant == "dropout":
+            fa.bwd(q, k, v, out, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, **drop)
+            mark(2)
+            return
+        for st in range(3):
+            fa.bwd(q, k, v, out, lse, do, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, stage=st)
+            mark(2 + st)
 
     for _ in range(args.warmup):
         step()
@@ -394,11 +428,11 @@ def run_ours(args):
                     stream.wait_event(downloaded[i - 2])  # step i-2's gradients have left this output set
                 ins = dev_in[x]
                 if fwd_only:
-                    fa.fwd(ins[0], ins[1], ins[2], causal=w.causal, out=dev_out[x][0], lse=dev_lse[x])
+                    fwd_call(ins[0], ins[1], ins[2], dev_out[x][0], dev_lse[x])
                 else:
-                    o_, l_ = fa.fwd(ins[0], ins[1], ins[2], causal=w.causal, out=dev_o[x], lse=dev_lse[x])
+                    o_, l_ = fwd_call(ins[0], ins[1], ins[2], dev_o[x], dev_lse[x])
                     fa.bwd(ins[0], ins[1], ins[2], o_, l_, ins[3], causal=w.causal, dq=dev_out[x][0],
-                           dk=dev_out[x][1], dv=dev_out[x][2], workspace=ws)
+                           dk=dev_out[x][1], dv=dev_out[x][2], workspace=ws, **drop)
                 computed[i].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(computed[i])
@@ -428,26 +462,33 @@ def run_ours(args):
     dom = max(per_kernel, key=per_kernel.get)
     dom_flops = flops_fwd if dom == "fa_fwd" else flops_bwd  # the backward's products all run in its main kernel
     achieved = dom_flops / (per_kernel[dom] / 1e3) / 1e12
-    traffic = recorded_traffic(dom, w.name)
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_source": "burst bf16 of %s" % peak_src,
+    traffic = recorded_traffic(dom, w.name) if variant == "plain" else None
+    # e4m3 products: the measured bf16 peak times the nominal e4m3/bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+    peak = peaks["bf16_tflops"] * (2.0 if variant == "fp8" else 1.0)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": ("burst bf16 of %s x 2 (nominal e4m3/bf16 ratio)" if variant == "fp8"
+                                else "burst bf16 of %s") % peak_src,
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_nominal_2250": achieved / NOMINAL_BF16_TFLOPS,
                 "algorithmic_flops_per_launch": dom_flops}
     kernels = {n: {"ms": per_kernel[n]} for n in names}
     kernels["fa_fwd"]["tflops"] = flops_fwd / (per_kernel["fa_fwd"] / 1e3) / 1e12
-    if not fwd_only:
+    if variant == "dropout":
+        kernels["fa_bwd"]["tflops"] = flops_bwd / (per_kernel["fa_bwd"] / 1e3) / 1e12
+        bwd_ms = per_kernel["fa_bwd"]
+    elif not fwd_only:
         kernels["fa_bwd_main"]["tflops"] = flops_bwd / (per_kernel["fa_bwd_main"] / 1e3) / 1e12
         bwd_ms = per_kernel["fa_bwd_pre"] + per_kernel["fa_bwd_main"] + per_kernel["fa_bwd_dq"]
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and variant == "plain":
         val, desc, threads, _ = oracle_sample(w, q, k, v, do, args.cpu_seconds)
         cpu = cpu_baseline_record(w, val, threads, desc)
     clocks = sampler.summary(t_host0, t_host1)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world), "roofline": roofline,
+            "dtype": "e4m3" if variant == "fp8" else "bf16", "data": "synthetic",
+            "config": variant_config(workload_config(w, world), variant), "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(names) * K, "clocks": clocks,
             "fwd_tflops": kernels["fa_fwd"]["tflops"],
             "fwd_frac_of_measured_peak": kernels["fa_fwd"]["tflops"] / peaks["bf16_tflops"],
