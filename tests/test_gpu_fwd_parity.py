@@ -104,3 +104,18 @@ def test_long_context_sampled_rows():
     q, k, v = make_workload_inputs(w)
     hs = all_heads(w.B, w.H)
     print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 8, 2), chunk=4))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_pages_accuracy_check(causal):
+    """The skill page's accuracy snippet (Workflow 1, Step 4) compares flash attention with standard attention
+    in fp16 on (batch 1, heads 8, seqlen 512, headdim 64) and expects a maximum absolute difference below 1e-3;
+    the same check against the fp64 oracle."""
+    q, k, v = make_inputs(1, 512, 512, 8, 64, "f16", 1158)
+    out, _ = fa.fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    heads = all_heads(1, 8)
+    o_ref, _ = oracle_fwd(q, k, v, causal, None, heads)
+    err = float(np.abs(gather_rows(out, heads) - o_ref).max())
+    print("max abs diff %.3e" % err)
+    assert err < 1e-3
