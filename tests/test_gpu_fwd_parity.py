@@ -106,16 +106,17 @@ def test_long_context_sampled_rows():
     print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 8, 2), chunk=4))
 
 
-@pytest.mark.parametrize("causal", [False, True])
-def test_pages_accuracy_check(causal):
+def test_pages_accuracy_check():
     """The skill page's accuracy snippet (Workflow 1, Step 4) compares flash attention with standard attention
-    in fp16 on (batch 1, heads 8, seqlen 512, headdim 64) and expects a maximum absolute difference below 1e-3;
-    the same check against the fp64 oracle."""
+    (no mask) in fp16 on (batch 1, heads 8, seqlen 512, headdim 64) and expects a maximum absolute difference
+    below 1e-3; the same check against the fp64 oracle. (With a causal mask the first rows average few values
+    of |v| up to ~4, where half an fp16 ulp is already ~1e-3: those rows are held to the bounds of the parity
+    tests above, which include the output rounding.)"""
     q, k, v = make_inputs(1, 512, 512, 8, 64, "f16", 1158)
-    out, _ = fa.fwd(q, k, v, causal=causal)
+    out, _ = fa.fwd(q, k, v, causal=False)
     torch.cuda.synchronize()
     heads = all_heads(1, 8)
-    o_ref, _ = oracle_fwd(q, k, v, causal, None, heads)
+    o_ref, _ = oracle_fwd(q, k, v, False, None, heads)
     err = float(np.abs(gather_rows(out, heads) - o_ref).max())
     print("max abs diff %.3e" % err)
     assert err < 1e-3
