@@ -73,6 +73,11 @@ CASES = [
     (1, 300, 300, 2, 1, 64, True, (-1, -1), "f16", 0.5),
     (2, 200, 129, 3, 3, 64, False, (-1, -1), "bf16", 0.2),
     (1, 640, 640, 4, 2, 128, True, (200, 0), "f16", 0.15),
+    (1, 1, 1, 1, 1, 128, False, (-1, -1), "bf16", 0.5),          # one query, one key
+    (1, 129, 1, 2, 2, 128, True, (-1, -1), "f16", 0.2),          # one key: rows 0..127 see none
+    (1, 517, 333, 2, 1, 64, True, (100, -1), "bf16", 0.3),       # MQA, left bound, rows without keys
+    (2, 384, 384, 8, 1, 128, True, (-1, -1), "bf16", 0.1),       # MQA, group 8: the backward walks 8 heads
+    (1, 256, 300, 2, 2, 64, False, (-1, -1), "f16", 0.9),        # t = 230: scale 1/(1 - 230/256)
 ]
 
 

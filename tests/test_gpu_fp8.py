@@ -79,6 +79,9 @@ CASES = [
     (1, 700, 700, 4, 1, False, (128, 128), False),
     (1, 1000, 1000, 2, 2, True, (256, 0), True),
     (1, 517, 333, 2, 1, True, (100, -1), False),   # rows without keys
+    (1, 1, 1, 1, 1, False, (-1, -1), False),       # one query, one key
+    (1, 5, 1000, 2, 2, True, (-1, -1), True),      # short query block at the end of a long key range
+    (1, 1000, 5, 2, 1, True, (-1, -1), False),     # five keys: all but the last five rows see none
 ]
 
 
