@@ -179,7 +179,7 @@ def oracle_sample(w, q, k, v, do, seconds, seed=0):
     to64 = lambda x: x[0, :, 0, :].detach().to("cpu").double().numpy()[None]  # noqa: E731
     qh, kh, vh, doh = to64(q), to64(k), to64(v), to64(do)
     rng = np.random.default_rng(seed)
-    fwd_only = w.name.startswith("long")
+    fwd_only = not w.backward
 
     def flops(rows):
         keys = np.minimum(w.Sk, rows + (w.Sk - w.Sq) + 1) if w.causal else np.full(rows.shape, w.Sk)
@@ -216,7 +216,7 @@ def cpu_model():
 def cpu_baseline_record(w, value, threads, desc):
     """The oracle's sampled rate, the host it ran on, and the time the whole problem would take at that rate
     (an extrapolation, labelled as one)."""
-    full = w.fwd_flops() + (0 if w.name.startswith("long") else w.bwd_flops())
+    full = w.fwd_flops() + (w.bwd_flops() if w.backward else 0)
     return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
             "cpu_model": cpu_model(), "extrapolated_full_problem_s": full / (value * 1e12) if value > 0 else None}
 
@@ -260,7 +260,7 @@ L2_BYTES = 126 << 20
 
 def input_bytes(w):
     """Bytes one step reads as its inputs (q, k, v, and dO for a training step)."""
-    return (3 if w.name.startswith("long") else 4) * w.B * w.Sq * w.H * w.D * 2
+    return (4 if w.backward else 3) * w.B * w.Sq * w.H * w.D * 2
 
 
 def variant_config(cfg, variant):
@@ -275,7 +275,7 @@ def variant_config(cfg, variant):
 
 
 def workload_config(w, n):
-    kind = "forward" if w.name.startswith("long") else "training step (forward + recomputation backward)"
+    kind = "training step (forward + recomputation backward)" if w.backward else "forward"
     return {"workload": "%s %s: B=%d H=%d Sq=%d Sk=%d D=%d %s %s" % (
                 w.name, kind, w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, "causal" if w.causal else "non-causal"),
             "global_batch": w.B * n, "seq_len": w.Sq,
@@ -298,7 +298,7 @@ def run_ours(args):
     replicas.init("nccl" if world > 1 else "gloo")
     w = workload_from_args(args)
     variant = args.variant
-    fwd_only = w.name.startswith("long") or variant == "fp8"
+    fwd_only = not w.backward or variant == "fp8"
     seed = replicas.replica_seed(w.seed, rank)
     q, k, v, do = make_inputs(w.B, w.Sq, w.Sk, w.H, w.D, w.dtype, seed, w.sigma, "cuda", with_dout=True)
     out = torch.empty_like(q)

@@ -433,6 +433,7 @@ __global__ void __launch_bounds__(384, 1)
         // relieves the MUFU unit (8-bit inputs only, where the tensor work per tile is half).
         auto p_loop = [&](auto emu_tag) {
           constexpr bool kEmu = decltype(emu_tag)::value && L::kEmuEvery > 0;
+          constexpr int kEmuPeriod = L::kEmuEvery > 0 ? L::kEmuEvery : 1;  // never a zero divisor
           const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m_use, -m_use);
           uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -440,7 +441,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t x01 = f2_fma(f2_pack(s[c], s[c + 1]), sc2, nm2);
             const uint64_t x23 = f2_fma(f2_pack(s[c + 2], s[c + 3]), sc2, nm2);
             float p0, p1, p2, p3;
-            if (kEmu && (c / 4) % L::kEmuEvery == L::kEmuEvery - 1) {
+            if (kEmu && (c / 4) % kEmuPeriod == kEmuPeriod - 1) {
               exp2_poly2(x01, p0, p1);
               exp2_poly2(x23, p2, p3);
             } else {

@@ -33,6 +33,13 @@ def test_flop_figures_of_the_full_size_workloads():
     assert round(long_.fwd_flops() / 1e9) == 140739                 # ≈ 140,740 GFLOP
 
 
+def test_only_the_gpt_workload_is_a_training_step():
+    # the benchmark plan: tiny, small, mid and long context are forward passes (O and LSE); the GPT-style
+    # workload is a forward plus the recomputation backward
+    assert [n for n, w in WORKLOADS.items() if w.backward] == ["gpt"]
+    assert len([n for n in WORKLOADS if n.startswith("mid_")]) == 8
+
+
 def test_e4m3_inputs():
     g = torch.Generator()
     g.manual_seed(0)
