@@ -565,8 +565,8 @@ __global__ void __launch_bounds__(384, 1)
   } else {
     // ------------------------------------------------------------------ dQ warpgroup (warps 4-7)
     // Each dQ partial goes TMEM -> registers -> fp32 reductions into dQacc in L2. (Staging it in shared memory
-    // for a bulk reduction costs 64 KB of shared-memory traffic per tile, which this kernel cannot spare: the
-    // MMAs' operand reads already come close to the shared-memory bandwidth.)
+    // for a bulk reduce-add adds 64 KB of shared-memory traffic and a staging hand-off per tile, and measured
+    // slower at the 4x32x8192x128 workload.)
     if constexpr (L::kRegsDQ < 168) regs_dec<L::kRegsDQ>();
     const uint32_t quarter = warp - 4;
     const int r = quarter * 32 + lane;  // TMEM lane: head-dim index (D = 128) or query row (D = 64)
