@@ -413,6 +413,23 @@ def pin_dropout_keep_block(orc):
     assert np.array_equal(keep, np.array(kb["keep"], bool)), ("hand-derived keep block", keep.astype(int))
 
 
+def pin_dropout_counter_layout(orc):
+    # The published known answers reach only block (0, 0), where the row-block and key-block counter words are
+    # equal, so the layout itself (the reading of the dropout stream: word i mod 4, byte j mod 4 of the
+    # generator's output for counter (i / 4, j / 4, head number, offset) under key (seed low, seed high)) is
+    # checked against the generator, which the known answers pin separately, on a ragged 10 x 19 mask whose
+    # blocks have unequal row and key indices.
+    p, seed, offset, bh = 0.3, 0x0123456789ABCDEF, 5, 6
+    t = math.floor(256 * p + 0.5)
+    key = (seed & 0xFFFFFFFF, seed >> 32)
+    keep = orc.dropout_mask(p, seed, offset, bh, 10, 19)
+    for i in range(10):
+        for j in range(19):
+            word = orc.philox4x32_10((i // 4, j // 4, bh, offset), key)[i % 4]
+            expect = ((word >> (8 * (j % 4))) & 0xFF) >= t
+            assert keep[i, j] == expect, ("dropout counter layout", i, j)
+
+
 def pin_dropout_zero_is_plain(orc):
     r = _rng(16)
     q, k, v, do = (r.standard_normal((2, 7, 3)) for _ in range(4))
@@ -538,6 +555,6 @@ ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_s
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
             pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,
-            pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_zero_is_plain, pin_dropout_keep_rate,
-            pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences,
+            pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_counter_layout, pin_dropout_zero_is_plain,
+            pin_dropout_keep_rate, pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences,
             pin_value_linearity]

@@ -42,6 +42,12 @@ MUTANTS = {
     "dropout_counter_ignores_head": ("(uint32_t)(j >> 2), (uint32_t)bh, dr->offset};", "(uint32_t)(j >> 2), 0u, dr->offset};"),
     "dropout_dv_undropped": ("gv += G[r * Sk + j] * doh[i * D + d];", "gv += P[r * Sk + j] * doh[i * D + d];"),
     "dropout_dp_unmasked": ("dP[j] = z * acc;", "dP[j] = acc;"),
+    "dropout_counter_rows_keys_swapped": ("(uint32_t)(i >> 2), (uint32_t)(j >> 2), (uint32_t)bh, dr->offset};",
+                                          "(uint32_t)(j >> 2), (uint32_t)(i >> 2), (uint32_t)bh, dr->offset};"),
+    "dropout_offset_ignored": ("(uint32_t)(j >> 2), (uint32_t)bh, dr->offset};", "(uint32_t)(j >> 2), (uint32_t)bh, 0u};"),
+    "philox_key_words_swapped": ("uint32_t k0 = key[0], k1 = key[1];", "uint32_t k0 = key[1], k1 = key[0];"),
+    "window_right_off_by_one": ("if (m->right >= 0 && j > c + m->right) return 0;",
+                                "if (m->right >= 0 && j >= c + m->right) return 0;"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
