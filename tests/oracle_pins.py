@@ -111,6 +111,28 @@ def pin_key_permutation(orc):
     _close(l1, l2, what="perm LSE")
 
 
+def pin_masked_keys_have_no_influence(orc):
+    # A masked (query, key) pair takes no part in the row, whatever the key holds: rows 0-2 of a 6 x 6 problem
+    # see none of keys 3-5 (causal, and a window (1, 0) without the causal flag), which are replaced by vectors
+    # whose scores exceed every visible score of row 2 by far more than exp's range and by huge values. O, LSE,
+    # dQ and the rows' dK/dV contributions stay bit for bit the same, and keys 3-5 receive exactly zero.
+    r = _rng(40)
+    q, k, v, do = (r.standard_normal((1, 6, 3)) for _ in range(4))
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 3:] = 1e4 * q[0, 2]
+    v2[0, 3:] = 1e6
+    rows = np.array([[0, 1, 2]], np.int64)
+    for causal, window in ((True, (-1, -1)), (False, (1, 0))):
+        kw = dict(causal=causal, scale=0.5, rows=rows, window=window)
+        for a, b in zip(orc.fwd(q, k, v, **kw), orc.fwd(q, k2, v2, **kw)):
+            assert np.array_equal(a, b), ("masked keys change the forward", causal, window)
+        (dq1, dk1, dv1), (dq2, dk2, dv2) = orc.bwd(q, k, v, do, **kw), orc.bwd(q, k2, v2, do, **kw)
+        assert np.array_equal(dq1, dq2), ("masked keys change dQ", causal, window)
+        for g1, g2 in ((dk1, dk2), (dv1, dv2)):
+            assert np.array_equal(g1[:, :3], g2[:, :3]), ("masked keys change dK/dV", causal, window)
+            assert not g1[:, 3:].any() and not g2[:, 3:].any(), ("masked keys receive gradient", causal, window)
+
+
 def _loss(orc, q, k, v, do, causal, scale):
     out, _ = orc.fwd(q, k, v, causal=causal, scale=scale)
     return float(np.sum(out * do))
@@ -552,6 +574,7 @@ def pin_value_linearity(orc):
 
 
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
+            pin_masked_keys_have_no_influence,
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
             pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,

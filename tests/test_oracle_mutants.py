@@ -48,6 +48,7 @@ MUTANTS = {
     "philox_key_words_swapped": ("uint32_t k0 = key[0], k1 = key[1];", "uint32_t k0 = key[1], k1 = key[0];"),
     "window_right_off_by_one": ("if (m->right >= 0 && j > c + m->right) return 0;",
                                 "if (m->right >= 0 && j >= c + m->right) return 0;"),
+    "max_over_masked_scores": ("if (visible(i, j, mk) && s[j] > m) m = s[j];", "if (s[j] > m) m = s[j];"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
