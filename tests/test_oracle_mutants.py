@@ -49,6 +49,14 @@ MUTANTS = {
     "window_right_off_by_one": ("if (m->right >= 0 && j > c + m->right) return 0;",
                                 "if (m->right >= 0 && j >= c + m->right) return 0;"),
     "max_over_masked_scores": ("if (visible(i, j, mk) && s[j] > m) m = s[j];", "if (s[j] > m) m = s[j];"),
+    # the backward's rows are a listed subset: r indexes the list, i the absolute query row
+    "bwd_scores_row_r": ("row_scores(qh + i * D, kh, Sk, D, scale, s);", "row_scores(qh + r * D, kh, Sk, D, scale, s);"),
+    "bwd_mask_row_r": ("row_softmax(s, i, &mk, Pi);", "row_softmax(s, r, &mk, Pi);"),
+    "dp_dout_row_r": ("for (int64_t d = 0; d < D; ++d) acc += doh[i * D + d] * vh[j * D + d];",
+                      "for (int64_t d = 0; d < D; ++d) acc += doh[r * D + d] * vh[j * D + d];"),
+    "dk_q_row_r": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[r * D + d];"),
+    "dv_dout_row_r": ("gv += G[r * Sk + j] * doh[i * D + d];", "gv += G[r * Sk + j] * doh[r * D + d];"),
+    "bwd_dk_wrong_kv_head": ("double *dkh = dk + (h / group) * Sk * D;", "double *dkh = dk + (h % n_kv_heads) * Sk * D;"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
