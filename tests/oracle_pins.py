@@ -10,7 +10,8 @@ What pins it:
     V = ones gives O = 1 because every softmax row sums to 1;
   * hand-worked examples with their derivations (tests/golden/hand_examples.json);
   * invariants: joint permutation of (K, V) rows leaves a non-causal result unchanged; sum_j dK_j = 0 and
-    sum_j dV_j = sum_i dO_i per head;
+    sum_j dV_j = sum_i dO_i per head; keys hidden from a row by the mask have no influence on it, whatever
+    they hold (scores beyond exp's range included), and receive no gradient from it;
   * central finite differences of L = sum dO * O in fp64 on tiny shapes (the backward has no formula on
     the pages, so the gradient of the oracle's own forward is the definition it must match);
   * a library routine the definition reduces to: torch's scaled_dot_product_attention on the CPU in
@@ -25,7 +26,8 @@ What pins it:
     known-answer vectors and a keep block derived by hand from one of them (tests/golden/philox_dropout.json);
     dropout_p = 0 is the plain path; the keep rate matches 1 - t/256; O averaged over many seeds converges to
     the undropped O (the 1/(1 - p) rescale) with LSE unchanged; with V = I the output is P o Z itself; finite
-    differences with the mask held fixed;
+    differences with the mask held fixed (and heads numbered as in a larger batch); the counter layout of the
+    dropout stream applied to the pinned generator on blocks whose row and key indices differ;
   * linearity in V: sum_j v_j . dV_j equals the loss sum_i dO_i . O_i, with and without dropout.
 """
 import json
@@ -527,17 +529,20 @@ def pin_dropout_identity_values(orc):
 def pin_dropout_finite_differences(orc):
     r = _rng(19)
     h = 1e-6
-    for (nq, nkv, Sq, Sk, D, causal, window, p) in ((2, 1, 5, 6, 2, False, (-1, -1), 0.3),
-                                                     (2, 2, 6, 6, 3, True, (2, 0), 0.5)):
+    # the second case numbers its heads 7 and 3 (as head b * H + h of a larger batch would be): the backward must
+    # regenerate the forward's mask for those head numbers
+    for (nq, nkv, Sq, Sk, D, causal, window, p, heads) in ((2, 1, 5, 6, 2, False, (-1, -1), 0.3, None),
+                                                            (2, 2, 6, 6, 3, True, (2, 0), 0.5, [7, 3])):
+        hidx = None if heads is None else np.array(heads, np.int64)
         q = r.standard_normal((nq, Sq, D))
         k = r.standard_normal((nkv, Sk, D))
         v = r.standard_normal((nkv, Sk, D))
         do = r.standard_normal((nq, Sq, D))
         drop = (p, 77, 1)
-        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.7, window=window, dropout=drop)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=0.7, window=window, dropout=drop, head_index=hidx)
 
         def loss(qq, kk, vv):
-            out, _ = orc.fwd(qq, kk, vv, causal=causal, scale=0.7, window=window, dropout=drop)
+            out, _ = orc.fwd(qq, kk, vv, causal=causal, scale=0.7, window=window, dropout=drop, head_index=hidx)
             return float(np.sum(out * do))
 
         for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):

@@ -57,6 +57,10 @@ MUTANTS = {
     "dk_q_row_r": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[r * D + d];"),
     "dv_dout_row_r": ("gv += G[r * Sk + j] * doh[i * D + d];", "gv += G[r * Sk + j] * doh[r * D + d];"),
     "bwd_dk_wrong_kv_head": ("double *dkh = dk + (h / group) * Sk * D;", "double *dkh = dk + (h % n_kv_heads) * Sk * D;"),
+    "bwd_dropout_head_number_ignored": ("double z = dropout_z(dr, head_number(head_index, h), i, j);",
+                                        "double z = dropout_z(dr, h, i, j);"),
+    "fwd_dropout_flat_row": ("double pz = p[j] * dropout_z(dr, head_number(head_index, h), i, j);",
+                             "double pz = p[j] * dropout_z(dr, head_number(head_index, h), t, j);"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
