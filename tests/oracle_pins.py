@@ -26,7 +26,8 @@ What pins it:
     known-answer vectors and a keep block derived by hand from one of them (tests/golden/philox_dropout.json);
     dropout_p = 0 is the plain path; the keep rate matches 1 - t/256; O averaged over many seeds converges to
     the undropped O (the 1/(1 - p) rescale) with LSE unchanged; with V = I the output is P o Z itself; finite
-    differences with the mask held fixed (and heads numbered as in a larger batch); the counter layout of the
+    differences with the mask held fixed (and heads numbered as in a larger batch); hand-derived cases of the
+    probability's resolution t = floor(256 p + 1/2) and its rejections; the counter layout of the
     dropout stream applied to the pinned generator on blocks whose row and key indices differ;
   * linearity in V: sum_j v_j . dV_j equals the loss sum_i dO_i . O_i, with and without dropout.
 """
@@ -454,6 +455,35 @@ def pin_dropout_counter_layout(orc):
             assert keep[i, j] == expect, ("dropout counter layout", i, j)
 
 
+def pin_dropout_probability_resolution(orc):
+    # Hand-derived cases of the probability's resolution (tests/golden/philox_dropout.json): with V = I the
+    # output is P o Z, so every kept element is the undropped P times the case's scale 256 / (256 - t) and
+    # every dropped one is 0; probabilities that round to t = 256, or lie outside [0, 1), are rejected.
+    res = _golden_philox()["probability_resolution"]
+    r = _rng(41)
+    S = 32
+    q, k = 0.3 * r.standard_normal((1, S, S)), 0.3 * r.standard_normal((1, S, S))  # head dim S, so V = I fits
+    eye = np.eye(S)[None]
+    plain, _ = orc.fwd(q, k, eye, causal=False, scale=0.5)
+    for case in res["cases"]:
+        p = case["dropout_p"]
+        out, _ = orc.fwd(q, k, eye, causal=False, scale=0.5, dropout=(p, 11, 0))
+        keep = orc.dropout_mask(p, 11, 0, 0, S, S)
+        assert keep.any(), ("no element kept", p)
+        _close(out[0][keep], plain[0][keep] * case["scale"], what="kept scale at p = %g" % p)
+        assert not out[0][~keep].any(), ("dropped elements not zero", p)
+        if case["t"] == 0:
+            assert keep.all(), "t = 0 drops nothing"
+    for case in res["rejected"]:
+        for call in (lambda: orc.dropout_mask(case["dropout_p"], 11, 0, 0, S, S),
+                     lambda: orc.fwd(q, k, eye, causal=False, scale=0.5, dropout=(case["dropout_p"], 11, 0))):
+            try:
+                call()
+            except ValueError:
+                continue
+            raise AssertionError(("dropout probability accepted", case["dropout_p"]))
+
+
 def pin_dropout_zero_is_plain(orc):
     r = _rng(16)
     q, k, v, do = (r.standard_normal((2, 7, 3)) for _ in range(4))
@@ -583,6 +613,7 @@ ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_s
             pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
             pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,
-            pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_counter_layout, pin_dropout_zero_is_plain,
+            pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_counter_layout,
+            pin_dropout_probability_resolution, pin_dropout_zero_is_plain,
             pin_dropout_keep_rate, pin_dropout_unbiased, pin_dropout_identity_values, pin_dropout_finite_differences,
             pin_value_linearity]

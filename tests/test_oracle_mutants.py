@@ -61,6 +61,9 @@ MUTANTS = {
                                         "double z = dropout_z(dr, h, i, j);"),
     "fwd_dropout_flat_row": ("double pz = p[j] * dropout_z(dr, head_number(head_index, h), i, j);",
                              "double pz = p[j] * dropout_z(dr, head_number(head_index, h), t, j);"),
+    "dropout_threshold_truncated": ("int t = (int)floor(256.0 * p + 0.5);", "int t = (int)floor(256.0 * p);"),
+    "dropout_threshold_scale_255": ("int t = (int)floor(256.0 * p + 0.5);", "int t = (int)floor(255.0 * p + 0.5);"),
+    "dropout_threshold_accepts_256": ("return t <= 255 ? t : -1;", "return t <= 256 ? t : -1;"),
     "dk_transposed_index": ("gk += dS[r * Sk + j] * qh[i * D + d];", "gk += dS[r * Sk + j] * qh[j % Sq * D + d];"),
 }
 
