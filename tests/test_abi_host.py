@@ -120,3 +120,32 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(fa, "LIB_PATH", str(tmp_path / "libfa.so"))
     with pytest.raises(ImportError):
         fa.lib()
+
+
+@pytest.mark.parametrize("H,Hkv", [(6, 4), (6, 0), (0, 1), (4, -1)])
+def test_grouped_entry_points_reject_bad_head_groups(H, Hkv):
+    # H must be a positive multiple of Hkv >= 1; checked before anything touches a device
+    L = fa.lib()
+    assert L.fa_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, H, Hkv, 64, 0, -1, -1, 0.0, 1, None) == -1
+    assert L.fa_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, H, Hkv, 64, 0, -1, -1, 0.0,
+                       1, FAKE, 1 << 30, None) == -1
+    assert L.fa_fwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, H, Hkv, 64, 0, -1, -1, 0.0, 1, 0.1, 1, 0,
+                            None) == -1
+    assert L.fa_bwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, H, Hkv, 64, 0, -1, -1,
+                            0.0, 1, 0.1, 1, 0, FAKE, 1 << 30, None) == -1
+
+
+def test_noalloc_host_checks():
+    # sizes are validated, and problems whose workspace exceeds the fixed scratch rejected, before any device
+    # lookup (the scratch's address is only looked up for calls that can run)
+    L = fa.lib()
+    L.fa_bwd_noalloc.restype = ctypes.c_int
+    L.fa_bwd_noalloc.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + [ctypes.c_float, ctypes.c_int,
+                                                                               ctypes.c_void_p]
+    args = [FAKE] * 9
+    assert L.fa_bwd_noalloc(*args, 0, 128, 128, 1, 64, 1, 0.0, 1, None) == -1
+    assert L.fa_bwd_noalloc(*args, 1, 128, 128, 1, 64, 1, float("nan"), 1, None) == -1
+    assert L.fa_bwd_noalloc(*args, 1, 128, 128, 1, 96, 1, 0.0, 1, None) == -2
+    B, S, H, D = 1, 8192, 32, 128
+    assert fa.workspace_size(B, S, H, D) > (64 << 20)
+    assert L.fa_bwd_noalloc(*args, B, S, S, H, D, 1, 0.0, 1, None) == -5
