@@ -168,9 +168,26 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------ oracle leg
-def oracle_sample(w, q, k, v, do, seconds, seed=0):
-    """Time the fp64 oracle (forward + backward) on a bounded sample of query rows of one head of the workload.
-    Returns (TFLOP/s under the same FLOP convention, description, threads)."""
+CPU_SAMPLE_SEED = 0
+CPU_SAMPLE_FLOPS = 4e9  # about one second of the oracle on a 16-core host
+
+
+def oracle_rows(w):
+    """The oracle's sample, identical in both legs: a fixed number of query rows of head (b=0, h=0), chosen by
+    the workload alone (about CPU_SAMPLE_FLOPS of executed work, 16 to 256 rows) and drawn with a fixed seed."""
+    import numpy as np
+
+    per_row = (4 if not w.backward else 14) * w.D * w.Sk
+    n = int(max(16, min(256, w.Sq, CPU_SAMPLE_FLOPS // per_row)))
+    return np.sort(np.random.default_rng(CPU_SAMPLE_SEED).choice(w.Sq, n, replace=False)).astype(np.int64)
+
+
+def oracle_sample(w, q, k, v, do, reps=1):
+    """Time the fp64 oracle (forward, and backward for a training workload) ``reps`` times on the fixed row
+    sample of ``oracle_rows``. Returns (TFLOP/s under the benchmark's FLOP convention, TFLOP/s of the work the
+    oracle executes, description, threads, seconds). The oracle walks every key of a listed row (masked ones
+    too) in each of its loops: forward 4*D*Sk and backward 10*D*Sk FLOPs per row, while the convention counts
+    the visible keys only."""
     import numpy as np
 
     import oracle
@@ -178,28 +195,23 @@ def oracle_sample(w, q, k, v, do, seconds, seed=0):
     threads = len(os.sched_getaffinity(0))
     to64 = lambda x: x[0, :, 0, :].detach().to("cpu").double().numpy()[None]  # noqa: E731
     qh, kh, vh, doh = to64(q), to64(k), to64(v), to64(do)
-    rng = np.random.default_rng(seed)
     fwd_only = not w.backward
-
-    def flops(rows):
-        keys = np.minimum(w.Sk, rows + (w.Sk - w.Sq) + 1) if w.causal else np.full(rows.shape, w.Sk)
-        per = 4 if fwd_only else 14
-        return float(per * w.D * keys.sum())
-
-    def run(n):
-        rows = np.sort(rng.choice(w.Sq, n, replace=False)).astype(np.int64)[None]
-        t0 = time.perf_counter()
-        oracle.attn_fwd(qh, kh, vh, causal=w.causal, rows=rows)
+    rows = oracle_rows(w)
+    keys = np.minimum(w.Sk, rows + (w.Sk - w.Sq) + 1) if w.causal else np.full(rows.shape, w.Sk)
+    per = 4 if fwd_only else 14
+    algorithmic = float(per * w.D * keys.sum()) * reps
+    executed = float(per * w.D * w.Sk * len(rows)) * reps
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.attn_fwd(qh, kh, vh, causal=w.causal, rows=rows[None])
         if not fwd_only:
-            oracle.attn_bwd(qh, kh, vh, doh, causal=w.causal, rows=rows)
-        return time.perf_counter() - t0, flops(rows[0])
-
-    dt, fl = run(8)  # calibration
-    n = int(min(w.Sq, max(8, 8 * seconds / max(dt, 1e-3))))
-    dt, fl = run(n)
-    desc = "%d random query rows of head (b=0,h=0) of the %s workload, %s, fp64 oracle" % (
-        n, w.name, "forward only" if fwd_only else "forward + backward")
-    return fl / dt / 1e12, desc, threads, dt
+            oracle.attn_bwd(qh, kh, vh, doh, causal=w.causal, rows=rows[None])
+    dt = time.perf_counter() - t0
+    desc = ("%d query rows of head (b=0,h=0) of the %s workload drawn with seed %d, %s, fp64 oracle, %d run(s); the "
+            "oracle walks all %d keys of each row (executed %.3g TFLOP/s)" % (
+                len(rows), w.name, CPU_SAMPLE_SEED, "forward only" if fwd_only else "forward + backward", reps,
+                w.Sk, executed / dt / 1e12))
+    return algorithmic / dt / 1e12, executed / dt / 1e12, desc, threads, dt
 
 
 def cpu_model():
@@ -213,12 +225,13 @@ def cpu_model():
     return "unknown"
 
 
-def cpu_baseline_record(w, value, threads, desc):
+def cpu_baseline_record(w, value, executed, threads, desc):
     """The oracle's sampled rate, the host it ran on, and the time the whole problem would take at that rate
     (an extrapolation, labelled as one)."""
     full = w.fwd_flops() + (w.bwd_flops() if w.backward else 0)
     return {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
-            "cpu_model": cpu_model(), "extrapolated_full_problem_s": full / (value * 1e12) if value > 0 else None}
+            "executed_tflops": executed, "cpu_model": cpu_model(),
+            "extrapolated_full_problem_s": full / (value * 1e12) if value > 0 else None}
 
 
 # ------------------------------------------------------------------------------------------------ arms
@@ -232,21 +245,22 @@ def run_reference(args):
     w = workload_from_args(args)
     # One head of the workload's distribution is all the oracle sample reads (same recipe, generated on the CPU).
     q, k, v, do = make_inputs(1, w.Sq, w.Sk, 1, w.D, w.dtype, w.seed, w.sigma, "cpu", with_dout=True)
-    per_step_s = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    # Every step is one run of the same fixed sample the other arm's cpu_baseline leg times (oracle_rows).
     for _ in range(args.warmup):
-        oracle_sample(w, q, k, v, do, per_step_s / 4)
-    vals, secs = [], 0.0
+        oracle_sample(w, q, k, v, do)
+    vals, execs, secs = [], [], 0.0
     desc, threads = "", 0
-    for s in range(args.steps):
-        val, desc, threads, dt = oracle_sample(w, q, k, v, do, per_step_s / 4, seed=s + 1)
+    for _ in range(args.steps):
+        val, ex, desc, threads, dt = oracle_sample(w, q, k, v, do)
         vals.append(val)
+        execs.append(ex)
         secs += dt
     value = statistics.mean(vals)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": workload_config(w, 1),
-            "cpu_baseline": cpu_baseline_record(w, value, threads, desc),
+            "cpu_baseline": cpu_baseline_record(w, value, statistics.mean(execs), threads, desc),
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -482,8 +496,10 @@ def run_ours(args):
         bwd_ms = per_kernel["fa_bwd_pre"] + per_kernel["fa_bwd_main"] + per_kernel["fa_bwd_dq"]
     cpu = None
     if world == 1 and not args.no_cpu_baseline and variant == "plain":
-        val, desc, threads, _ = oracle_sample(w, q, k, v, do, args.cpu_seconds)
-        cpu = cpu_baseline_record(w, val, threads, desc)
+        _, _, _, _, t1 = oracle_sample(w, q, k, v, do)  # one untimed run (warm-up and calibration)
+        reps = int(max(1, min(30, round(args.cpu_seconds / max(t1, 1e-3)))))
+        val, ex, desc, threads, _ = oracle_sample(w, q, k, v, do, reps)
+        cpu = cpu_baseline_record(w, val, ex, threads, desc)
     clocks = sampler.summary(t_host0, t_host1)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -1,8 +1,8 @@
 """B200-native (sm_100a) exact IO-aware attention: a thin Python binding over the C ABI of ``libfa.so``.
 
 Every step of the computation runs in the library's CUDA kernels; this module only marshals arguments
-(PyTorch tensors -> device pointers, sizes and the current CUDA stream) and turns status codes into
-exceptions. There is no fallback: if the library is missing or fails to load, every call raises.
+(PyTorch tensors -> device pointers, sizes and a CUDA stream) and turns status codes into exceptions. There is
+no fallback: if the library is missing or fails to load, every call raises.
 
     fwd(q, k, v, causal=False, scale=None, window=(-1, -1)) -> (out, lse)
     bwd(q, k, v, out, lse, dout, causal=False, scale=None, window=(-1, -1)) -> (dq, dk, dv)
@@ -11,6 +11,10 @@ Layouts follow the C header (include/fa.h): q/out/dout [B, Sq, H, D], k/v [B, Sk
 grouped or multi-query K/V heads), fp16 or bf16, contiguous, on one CUDA device; lse is fp32 [B, H, Sq].
 ``scale=None`` means 1/sqrt(D); ``window=(left, right)`` limits each query to keys within left before and
 right after its aligned key (-1 = unbounded side).
+
+Every operand (inputs and caller-passed outputs alike) is checked against these shapes, dtypes and the
+device of ``q`` before anything is launched; a mismatch raises ``ValueError`` or ``TypeError``. Each call
+runs with ``q``'s device current and, unless a stream is given, on that device's current stream.
 """
 import ctypes
 import os
@@ -22,8 +26,8 @@ FA_F16, FA_BF16 = 0, 1
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED", -3: "FA_ERR_CUDA",
                 -4: "FA_ERR_TIMEOUT", -5: "FA_ERR_WORKSPACE"}
-EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_bwd", "fa_bwd_ex", "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size",
-           "fa_status_string", "fa_device_status")
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_fwd_dropout", "fa_bwd_dropout", "fa_bwd", "fa_bwd_ex",
+           "fa_bwd_stage", "fa_bwd_noalloc", "fa_bwd_workspace_size", "fa_status_string", "fa_device_status")
 
 _lib = None
 
@@ -44,17 +48,19 @@ def lib():
                           % LIB_PATH)
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    u32, u64 = ctypes.c_uint32, ctypes.c_uint64
     L.fa_fwd.restype = i
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_bwd_stage.restype = i
     L.fa_bwd_stage.argtypes = [i] + L.fa_bwd.argtypes
+    L.fa_bwd_noalloc.restype = i
+    L.fa_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [f, i, vp]
     L.fa_fwd_ex.restype = i
     L.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, vp]
     L.fa_fwd_fp8.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, f, f, f, vp]
-    u32, u64 = ctypes.c_uint32, ctypes.c_uint64
     L.fa_fwd_dropout.restype = i
     L.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, f, u64, u32, vp]
     L.fa_bwd_dropout.restype = i
@@ -76,6 +82,7 @@ def status_string(status):
     return lib().fa_status_string(int(status)).decode()
 
 
+# ------------------------------------------------------------------------------------------ operand checks
 def _dtype_code(t):
     import torch
 
@@ -86,20 +93,76 @@ def _dtype_code(t):
     raise TypeError("expected float16 or bfloat16, got %s" % t.dtype)
 
 
-def _stream_ptr(stream):
+def _check(name, t, dev, shape=None, dtype=None):
+    """``t`` must be a contiguous tensor on the CUDA device ``dev`` (and have ``shape`` / ``dtype`` if given)."""
+    d = getattr(t, "device", None)
+    if d is None or d.type != "cuda" or d != dev:
+        raise ValueError("%s must be a CUDA tensor on %s, got %s" % (name, dev, d))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def check_qkv(q, k, v, dtypes):
+    """Shapes of the inputs: q [B, Sq, H, D], k and v [B, Sk, Hkv, D] with Hkv >= 1 dividing H, one dtype (from
+    ``dtypes``) for all three, one CUDA device. Returns (B, Sq, Sk, H, Hkv, D, device)."""
+    dev = getattr(q, "device", None)
+    if dev is None or dev.type != "cuda":
+        raise ValueError("q must be a CUDA tensor, got device %s" % dev)
+    if len(q.shape) != 4:
+        raise ValueError("q must be a [B, Sq, H, D] tensor, got shape %s" % (tuple(q.shape),))
+    if q.dtype not in dtypes:
+        raise TypeError("q must be one of %s, got %s" % (tuple(str(x) for x in dtypes), q.dtype))
+    _check("q", q, dev)
+    B, Sq, H, D = q.shape
+    if len(k.shape) != 4 or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k must be [B=%d, Sk, Hkv, D=%d], got %s" % (B, D, tuple(k.shape)))
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError("the K/V head count %d must divide the query head count %d" % (Hkv, H))
+    _check("k", k, dev, dtype=q.dtype)
+    _check("v", v, dev, shape=k.shape, dtype=q.dtype)
+    return B, Sq, Sk, H, Hkv, D, dev
+
+
+def check_fwd_outputs(out, lse, B, Sq, H, D, dev, out_dtype):
     import torch
 
-    s = torch.cuda.current_stream() if stream is None else stream
+    _check("out", out, dev, shape=(B, Sq, H, D), dtype=out_dtype)
+    _check("lse", lse, dev, shape=(B, H, Sq), dtype=torch.float32)
+
+
+def check_bwd_operands(q, k, out, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Sq, H, D, dev):
+    check_fwd_outputs(out, lse, B, Sq, H, D, dev, q.dtype)
+    _check("dout", dout, dev, shape=q.shape, dtype=q.dtype)
+    _check("dq", dq, dev, shape=q.shape, dtype=q.dtype)
+    _check("dk", dk, dev, shape=k.shape, dtype=q.dtype)
+    _check("dv", dv, dev, shape=k.shape, dtype=q.dtype)
+    if workspace is not None:
+        _check("workspace", workspace, dev)
+        if workspace.numel() * workspace.element_size() < ws_bytes:
+            raise ValueError("workspace must hold at least %d bytes" % ws_bytes)
+
+
+def _stream(stream, dev):
+    import torch
+
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    if s.device != dev:
+        raise ValueError("stream is on %s but the tensors are on %s" % (s.device, dev))
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _check_bshd(name, t, dev):
-    if not t.is_cuda or t.device != dev:
-        raise ValueError("%s must be a CUDA tensor on %s" % (name, dev))
-    if t.dim() != 4 or not t.is_contiguous():
-        raise ValueError("%s must be a contiguous [B, S, H, D] tensor" % name)
+def _device(dev):
+    import torch
+
+    return torch.cuda.device(dev)
 
 
+# ------------------------------------------------------------------------------------------ entry points
 def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, window=(-1, -1), dropout_p=0.0, seed=0,
         offset=0):
     """Forward attention. Returns (out [B,Sq,H,D] in q's dtype, lse fp32 [B,H,Sq]).
@@ -108,22 +171,20 @@ def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, wind
     keyed by ``seed`` (64-bit) and ``offset`` (32-bit); the backward must get the same three values."""
     import torch
 
-    dev = q.device
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_bshd(n, t, dev)
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
-    Hkv = k.shape[2]
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, Hkv, D,
-            int(bool(causal)), int(window[0]), int(window[1]), float(0.0 if scale is None else scale), _dtype_code(q))
-    if dropout_p:
-        rc = lib().fa_fwd_dropout(*args, float(dropout_p), int(seed), int(offset), _stream_ptr(stream))
-    else:
-        rc = lib().fa_fwd_ex(*args, _stream_ptr(stream))
+    B, Sq, Sk, H, Hkv, D, dev = check_qkv(q, k, v, (torch.float16, torch.bfloat16))
+    with _device(dev):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+        check_fwd_outputs(out, lse, B, Sq, H, D, dev, q.dtype)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H, Hkv, D,
+                int(bool(causal)), int(window[0]), int(window[1]), float(0.0 if scale is None else scale),
+                _dtype_code(q))
+        if dropout_p:
+            rc = lib().fa_fwd_dropout(*args, float(dropout_p), int(seed), int(offset), _stream(stream, dev))
+        else:
+            rc = lib().fa_fwd_ex(*args, _stream(stream, dev))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_dropout" if dropout_p else "fa_fwd_ex")
     return out, lse
@@ -131,27 +192,21 @@ def fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, wind
 
 def fwd_fp8(q, k, v, causal=False, scale=None, descale=(1.0, 1.0, 1.0), out=None, lse=None, stream=None,
             window=(-1, -1)):
-    """Forward attention on float8_e4m3fn inputs (D = 128). The real inputs are q * descale[0], k * descale[1],
-    v * descale[2]. Returns (out bf16 [B,Sq,H,D], lse fp32 [B,H,Sq])."""
+    """Forward attention on float8_e4m3fn inputs (D = 64 or 128). The real inputs are q * descale[0],
+    k * descale[1], v * descale[2]. Returns (out bf16 [B,Sq,H,D], lse fp32 [B,H,Sq])."""
     import torch
 
-    dev = q.device
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_bshd(n, t, dev)
-        if t.dtype != torch.float8_e4m3fn:
-            raise TypeError("%s must be float8_e4m3fn, got %s" % (n, t.dtype))
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
-    if out is None:
-        out = torch.empty((B, Sq, H, D), dtype=torch.bfloat16, device=dev)
-    if lse is None:
-        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
-    if out.dtype != torch.bfloat16:
-        raise TypeError("out must be bfloat16")
-    rc = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk, H,
-                          k.shape[2], D, int(bool(causal)), int(window[0]), int(window[1]),
-                          float(0.0 if scale is None else scale), float(descale[0]), float(descale[1]),
-                          float(descale[2]), _stream_ptr(stream))
+    B, Sq, Sk, H, Hkv, D, dev = check_qkv(q, k, v, (torch.float8_e4m3fn,))
+    with _device(dev):
+        if out is None:
+            out = torch.empty((B, Sq, H, D), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+        check_fwd_outputs(out, lse, B, Sq, H, D, dev, torch.bfloat16)
+        rc = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Sq, Sk,
+                              H, Hkv, D, int(bool(causal)), int(window[0]), int(window[1]),
+                              float(0.0 if scale is None else scale), float(descale[0]), float(descale[1]),
+                              float(descale[2]), _stream(stream, dev))
     if rc != FA_OK:
         raise FAError(rc, "fa_fwd_fp8")
     return out, lse
@@ -169,42 +224,63 @@ def bwd(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=
     ``fa_bwd_stage`` in include/fa.h; a caller running the stages separately must pass the same workspace."""
     import torch
 
-    dev = q.device
-    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
-        _check_bshd(n, t, dev)
-    B, Sq, H, D = q.shape
-    Sk = k.shape[1]
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    ws_bytes = workspace_size(B, Sq, H, D)
-    if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    Hkv = k.shape[2]
-    sc = float(0.0 if scale is None else scale)
-    ws_args = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
-    if dropout_p:
-        if stage != -1:
-            raise ValueError("single backward stages are available for plain attention only")
-        rc = lib().fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, Hkv, D,
-                                  int(bool(causal)), int(window[0]), int(window[1]), sc, _dtype_code(q),
-                                  float(dropout_p), int(seed), int(offset), *ws_args)
-    elif stage == -1:
-        rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
-                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, Hkv, D, int(bool(causal)),
-                             int(window[0]), int(window[1]), sc, _dtype_code(q), *ws_args)
-    else:
-        if Hkv != H or tuple(window) != (-1, -1):
-            raise ValueError("single backward stages are available for plain attention only")
-        rc = lib().fa_bwd_stage(int(stage), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D,
-                                int(bool(causal)), sc, _dtype_code(q), *ws_args)
+    B, Sq, Sk, H, Hkv, D, dev = check_qkv(q, k, v, (torch.float16, torch.bfloat16))
+    if stage != -1 and (dropout_p or Hkv != H or tuple(window) != (-1, -1)):
+        raise ValueError("single backward stages are available for plain attention only")
+    with _device(dev):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        ws_bytes = workspace_size(B, Sq, H, D)
+        check_bwd_operands(q, k, out, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Sq, H, D, dev)
+        if workspace is None:
+            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        sc = float(0.0 if scale is None else scale)
+        ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr())
+        ws_args = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream, dev))
+        if dropout_p:
+            rc = lib().fa_bwd_dropout(*ptrs, B, Sq, Sk, H, Hkv, D, int(bool(causal)), int(window[0]), int(window[1]),
+                                      sc, _dtype_code(q), float(dropout_p), int(seed), int(offset), *ws_args)
+        elif stage == -1:
+            rc = lib().fa_bwd_ex(*ptrs, B, Sq, Sk, H, Hkv, D, int(bool(causal)), int(window[0]), int(window[1]), sc,
+                                 _dtype_code(q), *ws_args)
+        else:
+            rc = lib().fa_bwd_stage(int(stage), *ptrs, B, Sq, Sk, H, D, int(bool(causal)), sc, _dtype_code(q),
+                                    *ws_args)
     if rc != FA_OK:
         raise FAError(rc, "fa_bwd")
     return dq, dk, dv
 
 
-def device_status(reset=False):
-    """The device-side sticky status word (FA_OK, or FA_ERR_TIMEOUT after a kernel gave up on a wait)."""
-    return int(lib().fa_device_status(int(bool(reset))))
+def bwd_noalloc(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, stream=None):
+    """``fa_bwd_noalloc``: the plain backward with the library's fixed device scratch instead of a workspace
+    (problems up to FA_NOALLOC_SCRATCH_BYTES of workspace; see include/fa.h). Returns (dq, dk, dv)."""
+    import torch
+
+    B, Sq, Sk, H, Hkv, D, dev = check_qkv(q, k, v, (torch.float16, torch.bfloat16))
+    if Hkv != H:
+        raise ValueError("the no-alloc backward takes as many K/V heads as query heads")
+    with _device(dev):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        check_bwd_operands(q, k, out, lse, dout, dq, dk, dv, None, 0, B, Sq, H, D, dev)
+        rc = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Sk, H, D,
+                                  int(bool(causal)), float(0.0 if scale is None else scale), _dtype_code(q),
+                                  _stream(stream, dev))
+    if rc != FA_OK:
+        raise FAError(rc, "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
+def device_status(reset=False, device=None):
+    """The device-side sticky status word (FA_OK, or FA_ERR_TIMEOUT after a kernel gave up on a wait) of
+    ``device`` (default: the current device)."""
+    import torch
+
+    if device is None:
+        return int(lib().fa_device_status(int(bool(reset))))
+    with torch.cuda.device(device):
+        return int(lib().fa_device_status(int(bool(reset))))

@@ -137,7 +137,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int check_common(int B, int Sq, int Sk, int H, int D, float scale, int dtype) {
   if (B < 1 || Sq < 1 || Sk < 1 || H < 1 || D < 1) return FA_ERR_INVALID;
-  if (!isfinite(scale) || scale < 0.f) return FA_ERR_INVALID;
+  if (!isfinite(scale)) return FA_ERR_INVALID;
   if (dtype != FA_F16 && dtype != FA_BF16) return FA_ERR_INVALID;
   // TMA coordinates and the kernels' row indices are 32-bit; keep every extent far from overflow.
   const double elems_q = (double)B * Sq * H * D, elems_k = (double)B * Sk * H * D;
@@ -237,7 +237,7 @@ extern "C" {
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "ok";
-    case FA_ERR_INVALID: return "invalid argument (pointer, size, alignment, scale or dtype)";
+    case FA_ERR_INVALID: return "invalid argument (pointer, size, alignment, non-finite scale or dtype)";
     case FA_ERR_UNSUPPORTED: return "unsupported head dim or device (needs D in {64,128} on sm_100)";
     case FA_ERR_CUDA: return "CUDA call or kernel launch failed";
     case FA_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (device status)";

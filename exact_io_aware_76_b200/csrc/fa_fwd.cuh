@@ -21,7 +21,7 @@
 // The MMA issue order is S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ..., so while one warpgroup runs the
 // softmax of its tile the tensor core works on the other tile (ping-pong).
 //
-// Online softmax in the log2 domain: with c = scale*log2(e) and running max m (of s*c) and sum l,
+// Online softmax in the log2 domain: with c = scale*log2(e) (any sign) and running max m (of s*c) and sum l,
 //   m' = max(m, rowmax(S)*c);  p = 2^(S*c - m');  l' = l*2^(m-m') + rowsum(p);  O' = O*2^(m-m') + P V.
 // The O rescale is lazy: m only moves when the new max exceeds it by more than kRescaleLog2 (8, i.e. a
 // factor 256); otherwise p is computed against the stale m. Both O and l use the same m, so the final
@@ -324,6 +324,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t o_tmem = lane_base + 256 + t * D;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // Any finite scale: with c < 0 a masked score is +inf, so that s*c is -inf and its weight 0.
+    const bool neg_scale = p.scale_log2 < 0.f;
+    const float masked = neg_scale ? INFINITY : -INFINITY;
     // This row's visible keys (the causal mask and the window, clipped to [0, Sk)).
     const int row_lo = has_left ? row + off - p.win_left : 0;
     const int row_hi = has_right ? min(p.Sk - 1, row + off + right) : p.Sk - 1;
@@ -343,19 +346,33 @@ __global__ void __launch_bounds__(384, 1)
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (key0 + c < row_lo || key0 + c > row_hi) s[c] = -INFINITY;
+          if (key0 + c < row_lo || key0 + c > row_hi) s[c] = masked;
       }
-      // Row max: four independent chains of three-input maxima, then combined.
-      float mq[4] = {s[0], s[1], s[2], s[3]};
+      // The row's largest s*c: c times the largest score for c > 0, times the smallest for c < 0. Four
+      // independent chains of three-input maxima (minima), then combined.
+      float ext;
+      if (!neg_scale) {
+        float mq[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 4; c < 124; c += 8) {
-        mq[0] = fmax3(mq[0], s[c], s[c + 1]);
-        mq[1] = fmax3(mq[1], s[c + 2], s[c + 3]);
-        mq[2] = fmax3(mq[2], s[c + 4], s[c + 5]);
-        mq[3] = fmax3(mq[3], s[c + 6], s[c + 7]);
+        for (int c = 4; c < 124; c += 8) {
+          mq[0] = fmax3(mq[0], s[c], s[c + 1]);
+          mq[1] = fmax3(mq[1], s[c + 2], s[c + 3]);
+          mq[2] = fmax3(mq[2], s[c + 4], s[c + 5]);
+          mq[3] = fmax3(mq[3], s[c + 6], s[c + 7]);
+        }
+        ext = fmaxf(fmax3(mq[0], mq[1], s[124]), fmax3(mq[2], mq[3], fmax3(s[125], s[126], s[127])));
+      } else {
+        float mq[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < 124; c += 8) {
+          mq[0] = fmin3(mq[0], s[c], s[c + 1]);
+          mq[1] = fmin3(mq[1], s[c + 2], s[c + 3]);
+          mq[2] = fmin3(mq[2], s[c + 4], s[c + 5]);
+          mq[3] = fmin3(mq[3], s[c + 6], s[c + 7]);
+        }
+        ext = fminf(fmin3(mq[0], mq[1], s[124]), fmin3(mq[2], mq[3], fmin3(s[125], s[126], s[127])));
       }
-      const float mx = fmaxf(fmax3(mq[0], mq[1], s[124]), fmax3(mq[2], mq[3], fmax3(s[125], s[126], s[127])));
-      const float m_cand = fmaxf(m, mx * p.scale_log2);
+      const float m_cand = fmaxf(m, ext * p.scale_log2);
       // Warp-uniform decision: TMEM loads/stores below are warp-collective.
       const bool rescale = __any_sync(0xffffffffu, m_cand > m + kRescaleLog2);
       if (rescale) {

@@ -138,152 +138,6 @@ __global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns, int* w
   if (threadIdx.x == 0) *waited_ok = ok ? 1 : 0;
 }
 
-// Throughput probe: one thread per CTA issues `iters` back-to-back tcgen05 MMAs (K = 16 each) of one shape on
-// whatever the shared memory holds, then waits for them; cycles[blockIdx.x] receives the elapsed SM cycles.
-//   shape 0: SS, A K-major, B K-major   1: SS, A K-major, B MN-major   2: TS (A from TMEM), B MN-major
-//   shape 3: SS, A MN-major, B MN-major  4: TS, B K-major               5: SS, A MN-major, B K-major
-// MN-major operands use the 128-byte swizzle (the only form the kernels use).
-__global__ void __launch_bounds__(128, 1) selftest_mma_rate_kernel(int shape, int N, int iters, int swz,
-                                                                     long long* cycles, const uint8_t* src) {
-  using namespace fa;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 196608);  // operands read at most 192 KB
-  uint32_t* holder = reinterpret_cast<uint32_t*>(smem + 196608 + 48);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 196608 + 52);
-  volatile int* stop = reinterpret_cast<volatile int*>(smem + 196608 + 56);
-  if (threadIdx.x == 0) {
-    *stop = 0;
-    for (int i = 0; i < 5; ++i) mbar_init(bar + i, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (threadIdx.x < 32) {
-    tmem_alloc(holder, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tmem = *holder;
-  // Shapes 9 and 10 replay shape 8 while other warps add traffic: 9 = one thread streams 16 KB bulk copies from
-  // global memory into spare shared memory [200 KB, 216 KB); 10 = warps 2-3 stream TMEM loads/stores on the spare
-  // columns 448-511 of their lanes. Both stop when the MMA thread is done (or after a fixed number of rounds).
-  if (shape == 9 && threadIdx.x == 32) {
-    uint64_t* lbar = bar + 4;
-    int drain = 0;
-    for (int r = 0; r < 200000 && !*stop; ++r) {
-      mbar_arrive_expect_tx(lbar, 16384);
-      bulk_load(smem + 204800, src + (size_t)(r & 63) * 16384, 16384, lbar);
-      if (!mbar_wait(lbar, r & 1, &drain)) break;
-    }
-  }
-  if (shape == 10 && (threadIdx.x >> 5) >= 2) {
-    const uint32_t lane_base = tmem + (((threadIdx.x >> 5) * 32) << 16);
-    uint32_t rr[32];
-    for (int i = 0; i < 32; ++i) rr[i] = i;
-    for (int r = 0; r < 200000 && !*stop; ++r) {
-      tmem_ld_x32(lane_base + 448 + (r & 1) * 32, rr);
-      tmem_st_x32(lane_base + 448 + ((r + 1) & 1) * 32, rr);
-      tmem_st_wait();
-    }
-  }
-  if (threadIdx.x == 0) {
-    const uint32_t a = smem_u32(smem), b = smem_u32(smem + 32768);
-    // shape: 0 SS A-K B-K, 1 SS A-K B-MN, 2 TS B-MN, 3 SS A-MN B-MN, 4 TS B-K, 5 SS A-MN B-K.
-    const bool a_mn = (shape == 3 || shape == 5), b_mn = (shape == 1 || shape == 2 || shape == 3);
-    const bool ts = (shape == 2 || shape == 4);
-    const uint32_t idesc = idesc_f16(true, 128, N, a_mn, b_mn);
-    // Descriptors for the 8 K-steps are built before the timed loop so that the issue rate of the single
-    // thread does not limit the measurement (MN-major: 128-byte swizzle, K step 2048 B, blocks 16 KB apart).
-    uint64_t ad[8], bd[8];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      bd[kk] = b_mn ? sdesc_sw128(b + kk * 2048, 16384, 1024) : sdesc_sw128(b + (kk % 4) * 32, 16, 1024);
-      ad[kk] = a_mn ? sdesc_sw128(a + kk * 2048, 16384, 1024) : sdesc_sw128(a + (kk % 4) * 32, 16, 1024);
-    }
-    const long long t0 = clock64();
-    if (shape >= 8) {
-      // Same sequence on the kernel's own layout: K [0,32K), V [32K,64K), Q stages [64K,112K), dO stages
-      // [112K,160K), dS^T buffers [160K,192K); tiles rotate through the stages.
-      const uint32_t base = smem_u32(smem);
-      const uint32_t id64 = idesc_f16(true, 128, 64, false, false), id128 = idesc_f16(true, 128, 128, false, true);
-      const uint32_t idq = idesc_f16(true, 128, 64, true, true);
-      const uint64_t kk_desc = sdesc_sw128(base, 16, 1024), vk_desc = sdesc_sw128(base + 32768, 16, 1024);
-      const uint64_t kmn = sdesc_sw128(base, 16384, 1024);
-      const uint64_t qk = sdesc_sw128(base + 65536, 16, 1024), dok = sdesc_sw128(base + 114688, 16, 1024);
-      const uint64_t qmn = sdesc_sw128(base + 65536, 8192, 1024), domn = sdesc_sw128(base + 114688, 8192, 1024);
-      const uint64_t dsmn = sdesc_sw128(base + 163840, 16384, 1024);
-      for (int i = 0, t = 0; i < iters; i += 32, ++t) {
-        const uint32_t st = (t % 3) * 16384, x = t & 1;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + 256 + x * 64, sdesc_add(kk_desc, (kk / 4) * 16384 + (kk % 4) * 32),
-                  sdesc_add(qk, st + (kk / 4) * 8192 + (kk % 4) * 32), id64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + 384 + x * 64, sdesc_add(vk_desc, (kk / 4) * 16384 + (kk % 4) * 32),
-                  sdesc_add(dok, st + (kk / 4) * 8192 + (kk % 4) * 32), id64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tmem, tmem + 256 + x * 64 + kk * 8, sdesc_add(domn, st + kk * 2048), id128, 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tmem + 128, tmem + 384 + x * 64 + kk * 8, sdesc_add(qmn, st + kk * 2048), id128, 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + 384 + x * 64, sdesc_add(kmn, kk * 2048), sdesc_add(dsmn, x * 16384 + kk * 2048), idq, kk > 0);
-      }
-    } else if (shape >= 6) {
-      // The backward's per-tile sequence (D = 128, 64 queries): S^T and dP^T (8 + 8 SS, N = 64), dV and dK
-      // (4 + 4 TS, N = 128, B MN-major), dQ^T (8 SS, N = 64, A and B MN-major); shape 7 adds a commit after
-      // each group, as the kernel does. `iters` counts MMAs (32 per tile).
-      const uint32_t id64 = idesc_f16(true, 128, 64, false, false), id128 = idesc_f16(true, 128, 128, false, true);
-      const uint32_t idq = idesc_f16(true, 128, 64, true, true);
-      const uint64_t ka = sdesc_sw128(a, 16, 1024), qb = sdesc_sw128(b, 16, 1024);
-      const uint64_t amn = sdesc_sw128(a, 16384, 1024), bmn = sdesc_sw128(b, 8192, 1024);
-      for (int i = 0; i < iters; i += 32) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + 256, sdesc_add(ka, (kk / 4) * 16384 + (kk % 4) * 32), sdesc_add(qb, (kk / 4) * 8192 + (kk % 4) * 32), id64, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + 320, sdesc_add(ka, (kk / 4) * 16384 + (kk % 4) * 32), sdesc_add(qb, (kk / 4) * 8192 + (kk % 4) * 32), id64, kk > 0);
-        if (shape == 7) umma_commit(bar + 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_ts(tmem, tmem + 256 + kk * 8, sdesc_add(bmn, kk * 2048), id128, 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_ts(tmem + 128, tmem + 384 + kk * 8, sdesc_add(bmn, kk * 2048), id128, 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) umma_ss(tmem + 384, sdesc_add(amn, kk * 2048), sdesc_add(bmn, kk * 2048), idq, kk > 0);
-        if (shape == 7) {
-          umma_commit(bar + 2);
-          umma_commit(bar + 3);
-          umma_commit(bar + 4);
-        }
-      }
-    } else for (int i = 0; i < iters; i += 8) {
-      if (ts) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) umma_ts(tmem, tmem + 256 + kk * 8, bd[kk], idesc, 1);
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) umma_ss(tmem, ad[kk], bd[kk], idesc, 1);
-      }
-    }
-    umma_commit(bar);
-    mbar_wait(bar, 0, abort_flag);
-    cycles[blockIdx.x] = clock64() - t0;
-    *stop = 1;
-  }
-  tc_fence_before_sync();
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    tc_fence_after_sync();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 // 8-bit (e4m3) products with K = 128: variant 0: A [128][128] K-major, B [N][128] K-major (the S = Q K^T
 // form); variant 1: A [128][128] placed in TMEM four elements per column, B [128][N] MN-major (the O = P V form).
 __global__ void __launch_bounds__(128, 1)
@@ -435,27 +289,6 @@ extern "C" __attribute__((visibility("default"))) int fa_selftest_wait_timeout(u
   const int z = FA_OK;
   cudaMemcpyToSymbol(fa::g_device_status, &z, sizeof(int));
   return st;
-}
-
-// Runs the throughput probe on `ctas` CTAs (one per SM) and copies the per-CTA cycle counts to cycles_host.
-extern "C" __attribute__((visibility("default"))) int fa_selftest_mma_rate(int shape, int N, int iters, int swz,
-                                                                            int ctas, long long* cycles_host) {
-  if (shape < 0 || shape > 10 || (N != 64 && N != 128 && N != 256) || iters < 32 || (iters % 32) != 0 || ctas < 1 ||
-      ctas > 1024 || swz != 128)
-    return -1;
-  long long* d = nullptr;
-  uint8_t* src = nullptr;
-  if (cudaMalloc(&d, sizeof(long long) * ctas) != cudaSuccess) return -3;
-  if (cudaMalloc(&src, 64 * 16384) != cudaSuccess) return -3;
-  cudaMemset(src, 0, 64 * 16384);
-  const int smem = 221184 + 1024;  // operands up to 192 KB, bookkeeping at 192 KB, bulk-copy target 200-216 KB  // > half the SM's shared memory: one CTA per SM
-  cudaFuncSetAttribute(selftest_mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  selftest_mma_rate_kernel<<<ctas, 128, smem>>>(shape, N, iters, swz, d, src);
-  if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return -3;
-  cudaMemcpy(cycles_host, d, sizeof(long long) * ctas, cudaMemcpyDeviceToHost);
-  cudaFree(d);
-  cudaFree(src);
-  return 0;
 }
 
 // 8-bit layout check: variant 0 C = A B^T with A [128][128], B [N][128]; variant 1 C = A B with A [128][128]

@@ -254,6 +254,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Three-input minimum (one instruction on sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Packed pairs of fp32 (sm_100 executes add/fma on .f32x2 as one instruction for both halves).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -20,8 +20,8 @@
  *   - dtype: FA_F16 or FA_BF16 for every 16-bit tensor of a call (the pages: fp16/bf16 only, no fp32); the
  *     e4m3 forward (fa_fwd_fp8) takes 8-bit q, k, v and writes bf16.
  *   - D (head dim) in {64, 128}. B, H, Sq, Sk >= 1. Every pointer 16-byte aligned, device memory.
- *   - scale: 0.0f means 1/sqrt(D) (the pages' softmax_scale=None "Auto-scale"); any other finite value is
- *     used as given.
+ *   - scale: 0.0f (or -0.0f) means 1/sqrt(D) (the pages' softmax_scale=None "Auto-scale"); any other finite value,
+ *     negative ones included, is used as given; a non-finite scale is FA_ERR_INVALID.
  *   - causal != 0 applies the causal mask, bottom-right aligned when Sq != Sk: key j is visible to query i
  *     iff j <= i + (Sk - Sq). A query row that sees no key gets O = 0 and LSE = -inf.
  *   - lse[b,h,i] = ln sum_{j visible} exp(scale * q_i . k_j), fp32 (natural log, scale included).
@@ -56,7 +56,7 @@ typedef enum { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
 
 typedef enum {
   FA_OK = 0,
-  FA_ERR_INVALID = -1,     /* bad pointer, size, alignment, scale or dtype; nothing launched */
+  FA_ERR_INVALID = -1,     /* bad pointer, size, alignment, non-finite scale or dtype; nothing launched */
   FA_ERR_UNSUPPORTED = -2, /* head dim not in {64,128}, or the current device is not sm_100 */
   FA_ERR_CUDA = -3,        /* a CUDA call or kernel launch failed */
   FA_ERR_TIMEOUT = -4,     /* device status only: a kernel gave up on a bounded wait */

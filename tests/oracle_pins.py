@@ -240,6 +240,35 @@ def pin_sdpa_crosscheck(orc):
         _close(lse, torch.logsumexp(s, dim=-1).numpy(), what="logsumexp")
 
 
+def pin_negative_scale_sdpa(orc):
+    """Any finite scale is used as given, negative ones included: float64 CPU SDPA with the same negative
+    scale, causal and not. The scale of -200 puts the scores far beyond exp's range, so a row maximum taken
+    the wrong way round (the largest q.k instead of the largest scale * q.k) overflows and is caught."""
+    import torch
+
+    r = _rng(19)
+    for (Sq, Sk, D, causal, scale) in ((9, 9, 8, True, -0.7), (6, 11, 4, False, -0.35), (8, 8, 4, True, -200.0),
+                                       (5, 7, 8, False, -200.0)):
+        H = 2
+        q = r.standard_normal((H, Sq, D))
+        k = r.standard_normal((H, Sk, D))
+        v = r.standard_normal((H, Sk, D))
+        do = r.standard_normal((H, Sq, D))
+        mask = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq) if causal else None
+        o_ref, dq_ref, dk_ref, dv_ref = _sdpa(q, k, v, do, mask, scale)
+        out, lse = orc.fwd(q, k, v, causal=causal, scale=scale)
+        dq, dk, dv = orc.bwd(q, k, v, do, causal=causal, scale=scale)
+        big = max(1.0, abs(scale))
+        _close(out, o_ref, what="negative scale O")
+        _close(dq, dq_ref, tol=TOL * big, what="negative scale dQ")
+        _close(dk, dk_ref, tol=TOL * big, what="negative scale dK")
+        _close(dv, dv_ref, what="negative scale dV")
+        s_ = torch.tensor(np.einsum("hid,hjd->hij", q, k) * scale)
+        if mask is not None:
+            s_ = s_.masked_fill(~mask, float("-inf"))
+        _close(lse, torch.logsumexp(s_, dim=-1).numpy(), tol=TOL * big, what="negative scale logsumexp")
+
+
 def pin_causal_alignment(orc):
     r = _rng(10)
     # Sq < Sk: the last query sees every key, like the non-causal result; row i sees i + Sk - Sq + 1 keys.
@@ -610,7 +639,7 @@ def pin_value_linearity(orc):
 
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_first_causal_row, pin_rows_sum_to_one, pin_key_permutation,
             pin_masked_keys_have_no_influence,
-            pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck,
+            pin_finite_differences, pin_grad_invariants, pin_row_subset, pin_sdpa_crosscheck, pin_negative_scale_sdpa,
             pin_causal_alignment, pin_default_scale, pin_golden_hand_examples, pin_gqa_matches_repeated_kv,
             pin_gqa_and_window_finite_differences, pin_window_limits, pin_window_gqa_sdpa_crosscheck,
             pin_philox_known_answers, pin_dropout_keep_block, pin_dropout_counter_layout,

@@ -44,9 +44,17 @@ def fwd_call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Sq=128, Sk=128, H=1,
 @pytest.mark.parametrize("kw", [dict(q=None), dict(k=None), dict(v=None), dict(o=None), dict(lse=None),
                                 dict(q=MISALIGNED), dict(o=MISALIGNED), dict(lse=MISALIGNED), dict(B=0), dict(Sq=0),
                                 dict(Sk=-1), dict(H=0), dict(D=0), dict(scale=float("nan")),
-                                dict(scale=float("inf")), dict(scale=-0.5), dict(dtype=2)])
+                                dict(scale=float("inf")), dict(scale=float("-inf")), dict(dtype=2)])
 def test_fwd_rejects_invalid(kw):
     assert fwd_call(**kw) == -1
+
+
+@pytest.mark.parametrize("scale", [-0.5, -1e-30, -0.0, -300.0])
+def test_negative_scale_passes_validation(scale):
+    # any finite scale is used as given: a negative one gets past the argument checks and the call fails only
+    # at the (later) head-dim check, before anything touches a device
+    assert fwd_call(scale=scale, D=96) == -2
+    assert bwd_call(scale=scale, D=96) == -2
 
 
 @pytest.mark.parametrize("D", [32, 96, 256])

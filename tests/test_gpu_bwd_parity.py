@@ -26,15 +26,17 @@ def run_bwd(q, k, v, do, causal, scale=None):
     return out, lse, dq, dk, dv
 
 
-def check_full(q, k, v, do, causal, heads, scale=None, chunk=8):
+def check_full(q, k, v, do, causal, heads, scale=None, chunk=8, elementwise=False):
+    """Every row of ``heads``: each gradient's relative Frobenius error per head (and, with ``elementwise``,
+    element by element; see parity_util.check_grad)."""
     _, _, dq, dk, dv = run_bwd(q, k, v, do, causal, scale)
     info = []
     for c0 in range(0, len(heads), chunk):
         sub = heads[c0:c0 + chunk]
         dq_r, dk_r, dv_r = oracle_bwd(q, k, v, do, causal, scale, sub)
-        info.append(check_grad(gather_rows(dq, sub), dq_r, "dQ"))
-        info.append(check_grad(gather_rows(dk, sub), dk_r, "dK"))
-        info.append(check_grad(gather_rows(dv, sub), dv_r, "dV"))
+        info.append(check_grad(gather_rows(dq, sub), dq_r, "dQ", elementwise=elementwise))
+        info.append(check_grad(gather_rows(dk, sub), dk_r, "dK", elementwise=elementwise))
+        info.append(check_grad(gather_rows(dv, sub), dv_r, "dV", elementwise=elementwise))
     return info
 
 
@@ -44,7 +46,7 @@ def check_full(q, k, v, do, causal, heads, scale=None, chunk=8):
 ])
 def test_small_full(B, Sq, Sk, H, D, causal, dtype):
     q, k, v, do = make_inputs(B, Sq, Sk, H, D, dtype, seed=500 + Sq + D, with_dout=True)
-    print(check_full(q, k, v, do, causal, all_heads(B, H)))
+    print(check_full(q, k, v, do, causal, all_heads(B, H), elementwise=True))
 
 
 @pytest.mark.parametrize("D", [64, 128])
@@ -63,12 +65,22 @@ def test_mid_four_heads(D, dtype, sigma):
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_ragged_and_degenerate(B, Sq, Sk, H, D, causal, dtype):
     q, k, v, do = make_inputs(B, Sq, Sk, H, D, dtype, seed=900 + Sq + 3 * Sk + D, with_dout=True)
-    print(check_full(q, k, v, do, causal, all_heads(B, H)))
+    print(check_full(q, k, v, do, causal, all_heads(B, H), elementwise=True))
 
 
 def test_explicit_scale():
     q, k, v, do = make_inputs(1, 256, 256, 2, 128, "bf16", seed=31, with_dout=True)
     print(check_full(q, k, v, do, True, all_heads(1, 2), scale=0.2))
+
+
+@pytest.mark.parametrize("B,S,H,D,causal,scale,dtype", [
+    (1, 300, 2, 128, True, -0.09, "bf16"), (2, 257, 2, 64, False, -0.125, "f16"), (1, 200, 3, 128, False, -1.0, "f16"),
+])
+def test_negative_scale(B, S, H, D, causal, scale, dtype):
+    """Any finite softmax_scale is used as given, negative ones included (the largest s*c of a row is then c
+    times its smallest score)."""
+    q, k, v, do = make_inputs(B, S, S, H, D, dtype, seed=77 + S + D, with_dout=True)
+    print(check_full(q, k, v, do, causal, all_heads(B, H), scale=scale, elementwise=True))
 
 
 def test_gpt_workload_sampled_rows_and_invariants():
@@ -90,9 +102,9 @@ def test_gpt_workload_sampled_rows_and_invariants():
     for c0 in range(0, len(heads), 16):
         sub = heads[c0:c0 + 16]
         dq_r, dk_r, dv_r = oracle_bwd(q, k, v, do, True, None, sub, rows[c0:c0 + 16])
-        check_grad(gather_rows(dq, sub, rows[c0:c0 + 16]), dq_r, "dQ sampled rows")
-        check_grad(gather_rows(dk_m, sub), dk_r, "dK of sampled rows")
-        check_grad(gather_rows(dv_m, sub), dv_r, "dV of sampled rows")
+        check_grad(gather_rows(dq, sub, rows[c0:c0 + 16]), dq_r, "dQ sampled rows", per_head=False)
+        check_grad(gather_rows(dk_m, sub), dk_r, "dK of sampled rows", per_head=False)
+        check_grad(gather_rows(dv_m, sub), dv_r, "dV of sampled rows", per_head=False)
     # Invariants of the real run over every key: sum_j dK_j = 0, sum_j dV_j = sum_i dO_i (per head).
     sdk = dk.double().sum(dim=1)
     adk = dk.double().abs().sum(dim=1)

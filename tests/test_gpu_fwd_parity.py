@@ -76,10 +76,22 @@ def test_ragged_and_degenerate(B, Sq, Sk, H, D, causal, dtype):
     print(run_and_check(q, k, v, causal, None, 1.0))
 
 
-@pytest.mark.parametrize("scale", [0.05, 0.3])
+@pytest.mark.parametrize("scale", [0.05, 0.3, -0.05, -0.3])
 def test_explicit_scale(scale):
     q, k, v = make_inputs(1, 256, 256, 2, 64, "bf16", seed=3)
     print(run_and_check(q, k, v, True, scale, 1.0))
+
+
+@pytest.mark.parametrize("B,Sq,Sk,H,D,causal,scale,dtype", [
+    (1, 333, 200, 2, 128, True, -0.088, torch.bfloat16),   # rows without keys under a negative scale
+    (2, 300, 517, 3, 64, False, -1.5, torch.float16),     # large negative scale: exponents far below the max
+    (1, 1000, 1000, 2, 128, True, -0.2, torch.float16),   # many key tiles: the running extremum moves
+])
+def test_negative_scale(B, Sq, Sk, H, D, causal, scale, dtype):
+    """Any finite scale is used as given: with scale < 0 the row maximum of s * scale is scale times the
+    row's smallest score, and masked scores must carry no weight either way."""
+    q, k, v = make_inputs(B, Sq, Sk, H, D, dtype, seed=41 + Sq + D)
+    print(run_and_check(q, k, v, causal, scale, 1.0))
 
 
 def test_single_key_closed_form():

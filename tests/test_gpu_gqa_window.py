@@ -32,6 +32,8 @@ CASES = [
     (1, 517, 333, 2, 1, 64, True, (100, -1), "f16"),        # left bound only, rows without keys
     (1, 400, 400, 2, 2, 128, False, (-1, 40), "bf16"),      # right bound only
     (2, 640, 640, 6, 3, 128, True, (300, 0), "bf16"),       # GQA + window
+    (1, 1000, 1000, 4, 2, 64, True, (256, 256), "bf16"),    # the skill page's call as written: causal + (256, 256)
+    (1, 517, 700, 2, 2, 128, True, (100, 50), "f16"),       # causal with a positive right bound (capped at 0)
 ]
 
 
