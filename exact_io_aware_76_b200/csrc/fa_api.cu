@@ -7,10 +7,12 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd128.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
 
+using fa::Bwd128Smem;
 using fa::BwdParams;
 using fa::BwdSmem;
 using fa::FwdParams;
@@ -176,7 +178,8 @@ struct BwdLayout {
   int sq_pad;
 };
 
-// Workspace: fp32 dQ accumulator [B,H,Sq_pad,D], then D_i [B,H,Sq_pad], then LSE_i*log2(e) [B,H,Sq_pad].
+// Workspace: fp32 dQ accumulator (B*H*Sq_pad*D floats: [B,H,Sq_pad,64] for head dim 64, [B,H,Sq_pad/4,128,4]
+// for head dim 128), then D_i [B,H,Sq_pad], then LSE_i*log2(e) [B,H,Sq_pad].
 BwdLayout bwd_layout(int B, int Sq, int H, int D) {
   BwdLayout l;
   l.sq_pad = (Sq + 127) / 128 * 128;
@@ -195,26 +198,41 @@ int grid_for(long long work, int per_block, int dev) {
   return (int)(g < 1 ? 1 : g);
 }
 
-// stage -1: all three launches; 0: preprocess; 1: main; 2: dQ conversion.
+// stage -1: all three launches; 0: preprocess; 1: main; 2: dQ conversion. Head dim 128 runs the 128-query-tile
+// main kernel (fa_bwd128.cuh) and the matching dQ conversion (query-quad accumulator layout); head dim 64 the
+// kernel of fa_bwd.cuh.
 template <int D, bool BF16, bool CAUSAL, bool DROP = false>
 int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& tdo, const BwdParams& p, int dev, cudaStream_t stream) {
   static bool attr_done[kMaxDevices] = {};
-  auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL, DROP>;
-  int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
-  if (rc) return rc;
   if (stage < 0 || stage == 0) {
     const long long rows = (long long)p.B * p.H * p.Sq_pad;
     fa::fa_bwd_pre_kernel<D, BF16><<<grid_for(rows, 8, dev), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
-    kern<<<(unsigned)(p.n_kblk * p.B * p.Hkv), BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    const unsigned grid = (unsigned)(p.n_kblk * p.B * p.Hkv);
+    if constexpr (D == 128) {
+      auto kern = fa::fa_bwd_main128_kernel<BF16, CAUSAL, DROP>;
+      int rc = ensure_smem_attr(kern, Bwd128Smem::kAlloc, dev, attr_done);
+      if (rc) return rc;
+      kern<<<grid, Bwd128Smem::kThreads, Bwd128Smem::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    } else {
+      auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL, DROP>;
+      int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
+      if (rc) return rc;
+      kern<<<grid, BwdSmem<D>::kThreads, BwdSmem<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 2) {
-    const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;
-    fa::fa_bwd_dq_kernel<D, BF16><<<grid_for(n8, 256, dev), 256, 0, stream>>>(p);
+    if constexpr (D == 128) {
+      const long long n = (long long)p.B * p.H * (p.Sq_pad / 4) * 32;
+      fa::fa_bwd_dq128_kernel<BF16><<<grid_for(n, 256, dev), 256, 0, stream>>>(p);
+    } else {
+      const long long n8 = (long long)p.B * p.Sq * p.H * D / 8;
+      fa::fa_bwd_dq_kernel<D, BF16><<<grid_for(n8, 256, dev), 256, 0, stream>>>(p);
+    }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -403,7 +421,7 @@ static int bwd_impl(int stage, const void* q, const void* k, const void* v, cons
   if ((rc = current_device(&dev))) return rc;
   if (scale == 0.f) scale = 1.f / sqrtf((float)D);
 
-  const int bq = (D == 128) ? BwdSmem<128>::kBQ : BwdSmem<64>::kBQ;
+  const int bq = (D == 128) ? Bwd128Smem::kBQ : BwdSmem<64>::kBQ;  // query rows per tile of the main kernel
   CUtensorMap tq, tk, tv, tdo;
   if ((rc = make_bshd_map(&tq, q, B, Sq, H, D, dtype, bq))) return rc;
   if ((rc = make_bshd_map(&tdo, dout, B, Sq, H, D, dtype, bq))) return rc;
