@@ -73,7 +73,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [B, S, H, D] tensor of 16-bit (dtype FA_F16/FA_BF16) or 8-bit (dtype -1: e4m3 bytes) elements; box = one
-// 128-byte swizzle row of head-dim elements x 1 head x `rows` rows.
+// 128-byte swizzle row of head-dim elements x 1 head x `rows` rows. (For e4m3 at D = 64 the box is wider than the
+// head dim: the copy engine fills elements 64..127 of each row with zeros.)
 constexpr int kDtypeE4M3 = -1;
 // Host-side cache of encoded tensor maps: a training loop passes the same buffers call after call, and a map
 // depends only on the arguments below, so an identical key means an identical map. Small and round-robin; a
@@ -360,7 +361,6 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* ls
     return FA_ERR_INVALID;
   int rc = check_common(B, Sq, Sk, H, D, scale, FA_BF16);
   if (rc) return rc;
-  if (D != 128) return FA_ERR_UNSUPPORTED;  // an e4m3 row of 64 elements is only 64 bytes
   int dev = 0;
   if ((rc = current_device(&dev))) return rc;
   if (scale == 0.f) scale = 1.f / sqrtf((float)D);
@@ -387,6 +387,9 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* ls
   p.v_descale = v_descale;
   p.drop_t = 0;
   p.drop_k0 = p.drop_k1 = p.drop_off = 0;
+  if (D == 64)
+    return causal ? launch_fwd<64, true, true, true>(tq, tk, tv, p, dev, stream)
+                  : launch_fwd<64, true, false, true>(tq, tk, tv, p, dev, stream);
   return causal ? launch_fwd<128, true, true, true>(tq, tk, tv, p, dev, stream)
                 : launch_fwd<128, true, false, true>(tq, tk, tv, p, dev, stream);
 }

@@ -16,7 +16,8 @@
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go to the softmax warpgroups)
 // Registers: 384 threads x 168 at launch; setmaxnreg moves the third warpgroup to 88 and the two softmax
 // warpgroups to 208 (2*128*208 + 128*88 = 64512 = 384*168), enough to hold a full 128-column S row.
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D). P_t overwrites the first 64
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+N), O1 [256+N,256+2N) (N = D, or 128 for e4m3 at D = 64).
+// P_t overwrites the first 64
 // (16-bit P) or 32 (e4m3 P) columns of S_t and is the A operand of the PV MMA read straight from TMEM.
 // The MMA issue order is S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ..., so while one warpgroup runs the
 // softmax of its tile the tensor core works on the other tile (ping-pong).
@@ -56,12 +57,17 @@ template <int D, bool kFP8 = false>
 struct FwdSmem {
   static constexpr int kBM = 128, kBN = 128, kNQ = 2;
   static constexpr int kElem = kFP8 ? 1 : 2;                      // bytes per input element
-  static constexpr int kChunks = D * kElem / 128;                 // 128-byte column chunks per row
+  // 128-byte column chunks per row: an e4m3 row of 64 head-dim elements is 64 bytes, so its tile keeps one whole
+  // 128-byte swizzle row per key, the copy engine filling head dims 64..127 with zeros.
+  static constexpr int kChunks = (D * kElem + 127) / 128;
   static constexpr int kChunkElems = 128 / kElem;                 // elements per 128-byte chunk
-  static constexpr int kTileBytes = 128 * D * kElem;              // one 128-row tile
+  static constexpr int kTileBytes = 128 * kChunks * 128;          // one 128-row tile
   static constexpr int kStages = (kTileBytes >= 32768) ? 2 : 4;   // K/V ring depth
   static constexpr int kKSteps = D * kElem / 32;                  // MMA steps over the head dim (32 B each)
   static constexpr int kPCols = kFP8 ? 32 : 64;                   // TMEM columns of a packed P row
+  // O accumulator columns = N of the P V product: the head dim, except e4m3 at D = 64, whose V rows are whole
+  // 128-element swizzle rows (the zero-filled half included): N = 128 there, the upper 64 columns stay 0.
+  static constexpr int kON = (kFP8 && D == 64) ? 128 : D;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kNQ * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_qk = kFP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(kBF16, 128, 128, false, false);
-      constexpr uint32_t idesc_pv = kFP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(kBF16, 128, D, false, true);
+      constexpr uint32_t idesc_pv = kFP8 ? idesc_e4m3(128, L::kON, false, true) : idesc_f16(kBF16, 128, D, false, true);
       // Base descriptors are built once; every MMA below adds a compile-time byte offset to one of them
       // (building a descriptor per instruction would make this single issuing thread the bottleneck).
       const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(384, 1)
       // P), B = V_j MN-major (as many 128-byte key rows per instruction; 64-wide head-dim blocks 16 KB apart).
       // Issued in two halves of 64 keys (with kSplitP the softmax publishes P of keys 0..63 first).
       auto issue_pv = [&](int t, int s, bool acc, int half) {
-        const uint32_t o_tmem = tmem + 256 + t * D;
+        const uint32_t o_tmem = tmem + 256 + t * L::kON;
         const uint32_t p_tmem = tmem + t * 128;
         const uint64_t b0 = sdesc_add(v_desc, s * L::kTileBytes);
         constexpr int kKeys = kFP8 ? 32 : 16;  // keys per instruction
@@ -321,7 +327,7 @@ __global__ void __launch_bounds__(384, 1)
     const int nt = n_kv[t];
     const uint32_t lane_base = tmem + ((quarter * 32) << 16);
     const uint32_t s_tmem = lane_base + t * 128;
-    const uint32_t o_tmem = lane_base + 256 + t * D;
+    const uint32_t o_tmem = lane_base + 256 + t * L::kON;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // Any finite scale: with c < 0 a masked score is +inf, so that s*c is -inf and its weight 0.

@@ -108,8 +108,8 @@ FA_API int fa_fwd_dropout(const void* q, const void* k, const void* v, void* out
  * input must be float8_e4m3fn"). q, k, v hold e4m3 bytes ([B,Sq,H,D] and [B,Sk,Hkv,D]); their real values are
  * the e4m3 values times q_descale, k_descale and v_descale (positive finite per-tensor factors; 1 for plain
  * e4m3 inputs). out is bf16 [B,Sq,H,D], lse fp32 [B,H,Sq]. The probabilities enter the P V product rounded to
- * e4m3 (round to nearest, saturating), so O carries up to 2^-4 relative error per probability term. D must be
- * 128 (FA_ERR_UNSUPPORTED otherwise). Heads, window and scale as in fa_fwd_ex.
+ * e4m3 (round to nearest, saturating), so O carries up to 2^-4 relative error per probability term. D in
+ * {64, 128} (FA_ERR_UNSUPPORTED otherwise). Heads, window and scale as in fa_fwd_ex.
  */
 FA_API int fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
                       int H, int Hkv, int D, int causal, int window_left, int window_right, float scale,

@@ -100,7 +100,7 @@ def test_fwd_fp8_rejects_invalid(kw):
     assert fwd_fp8_call(**kw) == -1
 
 
-@pytest.mark.parametrize("D", [32, 64, 256])
+@pytest.mark.parametrize("D", [32, 96, 256])
 def test_fwd_fp8_unsupported_head_dim(D):
     assert fwd_fp8_call(D=D) == -2
 

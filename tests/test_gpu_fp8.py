@@ -96,14 +96,15 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("B,Sq,Sk,H,Hkv,causal,window,scaled", CASES)
-def test_fp8_forward_within_rounding_bound(B, Sq, Sk, H, Hkv, causal, window, scaled):
+def test_fp8_forward_within_rounding_bound(B, Sq, Sk, H, Hkv, causal, window, scaled, D):
     g = torch.Generator(device="cuda")
-    g.manual_seed(7000 + Sq + H)
-    q, dq_ = draw_e4m3((B, Sq, H, 128), g, "cuda", per_tensor_scale=scaled)
-    k, dk_ = draw_e4m3((B, Sk, Hkv, 128), g, "cuda", per_tensor_scale=scaled)
-    v, dv_ = draw_e4m3((B, Sk, Hkv, 128), g, "cuda", per_tensor_scale=scaled)
-    scale = 1.0 / math.sqrt(128)
+    g.manual_seed(7000 + Sq + H + D)
+    q, dq_ = draw_e4m3((B, Sq, H, D), g, "cuda", per_tensor_scale=scaled)
+    k, dk_ = draw_e4m3((B, Sk, Hkv, D), g, "cuda", per_tensor_scale=scaled)
+    v, dv_ = draw_e4m3((B, Sk, Hkv, D), g, "cuda", per_tensor_scale=scaled)
+    scale = 1.0 / math.sqrt(D)
     out, lse = fa.fwd_fp8(q, k, v, causal=causal, scale=scale, descale=(dq_, dk_, dv_), window=window)
     torch.cuda.synchronize()
     assert fa.device_status() == 0
@@ -145,15 +146,16 @@ def sparse_pm1(shape, nnz, g):
     return x.to(torch.float8_e4m3fn)
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("causal,window,dq_", [(False, (-1, -1), 1.0), (True, (-1, -1), 0.5),
                                                 (False, (64, 200), 2.0)])
-def test_fp8_forward_exact_when_probabilities_are_powers_of_two(causal, window, dq_):
+def test_fp8_forward_exact_when_probabilities_are_powers_of_two(causal, window, dq_, D):
     B, Sq, Sk, H = 1, 384, 640, 2
     g = torch.Generator(device="cuda")
-    g.manual_seed(7100 + int(causal))
-    q = sparse_pm1((B, Sq, H, 128), 4, g)
-    k = sparse_pm1((B, Sk, H, 128), 4, g)
-    v, dv_ = draw_e4m3((B, Sk, H, 128), g, "cuda")
+    g.manual_seed(7100 + int(causal) + D)
+    q = sparse_pm1((B, Sq, H, D), 4, g)
+    k = sparse_pm1((B, Sk, H, D), 4, g)
+    v, dv_ = draw_e4m3((B, Sk, H, D), g, "cuda")
     dk_ = 1.0
     scale = math.log(2.0) / (dq_ * dk_)
     out, lse = fa.fwd_fp8(q, k, v, causal=causal, scale=scale, descale=(dq_, dk_, dv_), window=window)
@@ -201,3 +203,32 @@ def test_fp8_full_size_sampled_rows(name, n_heads, per_head):
         assert np.all(err <= bd), "head (%d,%d): max err/bound %.3f" % (b, h, float((err / bd).max()))
         check_lse(gather_lse(lse, [(b, h)], [rows]), l_ref)
     print("max err/bound %.3f over %d heads" % (worst, len(heads)))
+
+
+def test_fp8_skill_page_workflow3_shape():
+    """The skill page's only FP8 call (Workflow 3, Step 3): [2, 4096, 32, 64] tensors cast to float8_e4m3fn,
+    causal. Every row of two heads and 8 sampled rows (first, last, both sides of a tile edge, random) of every
+    other head, against the oracle on the dequantized inputs under the rounding bound."""
+    B, S, H, D = 2, 4096, 32, 64
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7300)
+    q8, k8, v8 = (torch.randn((B, S, H, D), generator=g, device="cuda").to(torch.float8_e4m3fn) for _ in range(3))
+    out, lse = fa.fwd_fp8(q8, k8, v8, causal=True)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    scale = 1.0 / math.sqrt(D)
+    r = np.random.default_rng(12)
+    worst = 0.0
+    for (b, h) in all_heads(B, H):
+        full = (b, h) in ((0, 0), (1, 31))
+        rows = np.arange(S, dtype=np.int64) if full else \
+            np.array([0, S - 1, 127, 128] + list(r.choice(S, 4, replace=False)), np.int64)
+        qh, kh, vh = deq(q8, 1.0, b, h), deq(k8, 1.0, b, h), deq(v8, 1.0, b, h)
+        o_ref, l_ref = oracle.attn_fwd(qh[None], kh[None], vh[None], causal=True, scale=scale, rows=rows[None])
+        bd = bound(qh, kh, vh, True, scale, (-1, -1), rows) + half_ulp(o_ref[0], torch.bfloat16)
+        o = gather_rows(out, [(b, h)], [rows])[0]
+        err = np.abs(o - o_ref[0])
+        worst = max(worst, float((err / bd).max()))
+        assert np.all(err <= bd), "head (%d,%d): max err/bound %.3f" % (b, h, float((err / bd).max()))
+        check_lse(gather_lse(lse, [(b, h)], [rows]), l_ref)
+    print("max err/bound %.3f over %d heads" % (worst, B * H))
