@@ -257,7 +257,9 @@ __global__ void __launch_bounds__(512, 1)
         }
         umma_commit(&q_empty[s]);
         // dQ^T = K^T dS^T into RP (the compute warps have read this tile's dP^T): A = K MN-major (head dim
-        // contiguous), B = dS^T MN-major (queries contiguous), 16 keys (2048 bytes) per instruction.
+        // contiguous), B = dS^T MN-major (queries contiguous), 16 keys (2048 bytes) per instruction. (Issuing it
+        // before dK, so that its read-out overlaps dK, measured no faster: the dQ warps' reductions then meet
+        // the issue of dK.)
         {
           uint64_t a = k_mn, bd = ds_mn;
           opaque(a, bd);
@@ -448,10 +450,18 @@ __global__ void __launch_bounds__(512, 1)
                        reinterpret_cast<uint32_t*>(v + 64));
       tc_fence_before_sync();
       mbar_arrive(dq_empty);
-      // Four queries of this head-dim index per 16-byte reduction; a warp covers 512 contiguous bytes.
+      // Four queries of this head-dim index per 16-byte reduction; a warp covers 512 contiguous bytes. The
+      // reductions are paced (a short sleep after each): issued back to back they fill the memory-instruction
+      // queue of every SM sub-partition, and the MMA thread's tcgen05 instructions, which wait in the same queue,
+      // stall behind them (measured, alternating runs on one B200: main kernel 6.26 -> 5.64 ms at
+      // 4x32x8192x128, within 4% of a timing copy with no reductions at all). A tile's 64 KB need only ~15 bytes
+      // per cycle of the ~23 an SM sustains.
       float* base = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * (p.Sq_pad / 4) + q0 / 4) * 512 + d * 4;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) red_add_v4(base + static_cast<size_t>(c) * 512, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      for (int c = 0; c < 32; ++c) {
+        red_add_v4(base + static_cast<size_t>(c) * 512, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        __nanosleep(60);
+      }
     }
   }
 
