@@ -35,7 +35,7 @@ NOMINAL_BF16_TFLOPS = 2250.0
 _COMMON_SOURCES = ["exact_io_aware_76_b200/csrc/sm100.cuh", "exact_io_aware_76_b200/csrc/tmem_ldst.inc",
                    "exact_io_aware_76_b200/csrc/dropout.cuh"]
 KERNEL_SOURCES = {
-    "fa_bwd_main": ["exact_io_aware_76_b200/csrc/fa_bwd.cuh"] + _COMMON_SOURCES,
+    "fa_bwd_main": ["exact_io_aware_76_b200/csrc/fa_bwd128.cuh", "exact_io_aware_76_b200/csrc/fa_bwd.cuh"] + _COMMON_SOURCES,
     "fa_fwd": ["exact_io_aware_76_b200/csrc/fa_fwd.cuh"] + _COMMON_SOURCES,
 }
 
@@ -169,16 +169,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------------------ oracle leg
 CPU_SAMPLE_SEED = 0
-CPU_SAMPLE_FLOPS = 4e9  # about one second of the oracle on a 16-core host
+CPU_SAMPLE_FLOPS = 1.6e10  # under a second of the oracle on a 16-core host
 
 
 def oracle_rows(w):
     """The oracle's sample, identical in both legs: a fixed number of query rows of head (b=0, h=0), chosen by
-    the workload alone (about CPU_SAMPLE_FLOPS of executed work, 16 to 256 rows) and drawn with a fixed seed."""
+    the workload alone (about CPU_SAMPLE_FLOPS of executed work, 16 to 1024 rows) and drawn with a fixed seed."""
     import numpy as np
 
     per_row = (4 if not w.backward else 14) * w.D * w.Sk
-    n = int(max(16, min(256, w.Sq, CPU_SAMPLE_FLOPS // per_row)))
+    n = int(max(16, min(1024, w.Sq, CPU_SAMPLE_FLOPS // per_row)))
     return np.sort(np.random.default_rng(CPU_SAMPLE_SEED).choice(w.Sq, n, replace=False)).astype(np.int64)
 
 
@@ -192,7 +192,9 @@ def oracle_sample(w, q, k, v, do, reps=1):
 
     import oracle
 
-    threads = len(os.sched_getaffinity(0))
+    # The same OpenMP team size in every process that times the oracle: one thread per core this process may
+    # run on (torch, loaded first, may have set its own default in the shared OpenMP runtime).
+    threads = oracle.set_threads(len(os.sched_getaffinity(0)))
     to64 = lambda x: x[0, :, 0, :].detach().to("cpu").double().numpy()[None]  # noqa: E731
     qh, kh, vh, doh = to64(q), to64(k), to64(v), to64(do)
     fwd_only = not w.backward

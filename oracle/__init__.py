@@ -67,7 +67,13 @@ class Oracle:
         lib.oracle_philox4x32_10.argtypes = [ctypes.POINTER(u32), ctypes.POINTER(u32), ctypes.POINTER(u32)]
         lib.oracle_dropout_mask.restype = ctypes.c_int
         lib.oracle_dropout_mask.argtypes = [dbl, u64, u32, i64, i64, i64, ctypes.POINTER(ctypes.c_uint8)]
+        lib.oracle_set_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
         self.lib = lib
+
+    def set_threads(self, n):
+        """Use n OpenMP threads from the calling thread on (n < 1: unchanged); returns the count in effect."""
+        return int(self.lib.oracle_set_threads(int(n)))
 
     @staticmethod
     def _prep(q, k, v, rows):
@@ -198,6 +204,10 @@ def attn_bwd(q, k, v, dout, causal=False, scale=None, rows=None, window=(-1, -1)
 
 def philox4x32_10(ctr, key):
     return _get().philox4x32_10(ctr, key)
+
+
+def set_threads(n):
+    return _get().set_threads(n)
 
 
 def dropout_mask(dropout_p, seed, offset, bh, Sq, Sk):

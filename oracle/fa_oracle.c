@@ -48,9 +48,19 @@
  * Return value: 0 on success, -1 on an invalid argument (nothing written).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+
+/* Size of the OpenMP team that the parallel loops below use when called from this thread (n >= 1; n < 1 leaves
+ * it unchanged); returns the team size now in effect. Lets a caller that times the oracle in different
+ * processes use the same number of threads in each. */
+int oracle_set_threads(int n)
+{
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
+}
 
 /* ---------------------------------------------------------------------------------------- Philox4x32-10 */
 
