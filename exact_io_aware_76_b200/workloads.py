@@ -3,7 +3,8 @@
 The five workloads follow the benchmark plan: tiny (1x2x128x64 fp16 non-causal), small (2x8x512x64 fp16,
 causal and non-causal), mid (2x16x2048, D 64/128, fp16/bf16, causal, inputs scaled by 1 and 4), GPT-style
 training (4x32x8192x128 bf16 causal) and long context (1x32x131072x128 bf16 causal). The GPT-style step is a
-forward and a backward; the others are forward passes (O and LSE).
+forward and a backward; the others are forward passes (O and LSE). A sixth, skill_timing, is the timing shape
+of the skill page's Workflow 1 Step 4 (4x32x4096x64 fp16, non-causal), a forward pass.
 
 FLOP convention: forward 4*B*H*D*pairs (QK^T and PV), backward 10*B*H*D*pairs (five matrix products, the
 recomputation of QK^T included), where ``pairs`` counts only the (query, key) pairs the mask leaves visible.
@@ -74,6 +75,9 @@ for _D in (64, 128):
         for _sig in (1.0, 4.0):
             _n = "mid_d%d_%s_x%d" % (_D, _dt, int(_sig))
             WORKLOADS[_n] = Workload(_n, 2, 16, 2048, 2048, _D, _dt, True, _sig, 1002)
+# The skill page's own timing shape (Workflow 1, Step 4: flash_attn_func on (4, 4096, 32, 64) fp16 tensors,
+# no causal flag), as a forward workload for `bench.py --workload skill_timing`.
+WORKLOADS["skill_timing"] = Workload("skill_timing", 4, 32, 4096, 4096, 64, "f16", False, 1.0, 1005)
 
 
 def make_workload_inputs(w, device="cuda", with_dout=False):

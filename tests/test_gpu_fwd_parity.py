@@ -132,3 +132,33 @@ def test_pages_accuracy_check():
     err = float(np.abs(gather_rows(out, heads) - o_ref).max())
     print("max abs diff %.3e" % err)
     assert err < 1e-3
+
+
+# Mid-sized problems of between one and two waves of CTAs (148 < CTAs <= 296 on a 148-SM B200, a CTA taking 256
+# query rows of one (batch, head)): ragged lengths, Sq != Sk, grouped heads, a window, rows without keys and a
+# negative scale, each checked on every row of three heads and on sampled rows of all heads.
+@pytest.mark.parametrize("B,Sq,Sk,H,Hkv,D,causal,window,dtype,scale", [
+    (1, 5000, 5000, 10, 10, 128, True, (-1, -1), torch.bfloat16, None),   # 20 query blocks x 10 heads, ragged
+    (2, 2500, 3000, 8, 2, 64, True, (-1, -1), torch.float16, None),       # Sq != Sk, grouped heads
+    (1, 4100, 4100, 12, 4, 128, False, (300, 200), torch.float16, None),  # window, non-causal, ragged tail
+    (3, 1700, 900, 8, 8, 128, True, (-1, -1), torch.bfloat16, None),      # Sq > Sk: rows without keys
+    (1, 4000, 4000, 10, 10, 64, True, (-1, -1), torch.bfloat16, -0.1),    # negative scale
+])
+def test_mid_size_forward_shapes(B, Sq, Sk, H, Hkv, D, causal, window, dtype, scale):
+    n_units = ((Sq + 255) // 256) * B * H
+    assert 148 < n_units <= 296, n_units
+    g = torch.Generator(device="cuda")
+    g.manual_seed(600 + Sq + H)
+    from exact_io_aware_76_b200.inputs import draw
+    q = draw((B, Sq, H, D), dtype, g, "cuda")
+    k = draw((B, Sk, Hkv, D), dtype, g, "cuda")
+    v = draw((B, Sk, Hkv, D), dtype, g, "cuda")
+    out, lse = fa.fwd(q, k, v, causal=causal, scale=scale, window=window)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    hs = all_heads(B, H)
+    # every row of three heads, sampled rows of all heads
+    for heads, rows in ((hs[:1] + hs[len(hs) // 2:len(hs) // 2 + 1] + hs[-1:], None),
+                        (hs, sampled_rows(Sq, hs, 6, 9))):
+        o_ref, l_ref = oracle_fwd(q, k, v, causal, scale, heads, rows, window=window)
+        print(check_out(gather_rows(out, heads, rows), o_ref, dtype), check_lse(gather_lse(lse, heads, rows), l_ref))
