@@ -270,7 +270,10 @@ __global__ void __launch_bounds__(512, 1)
         umma_commit(dq_full);
         umma_commit(ds_empty);
         if (more) {
-          if (!mbar_wait(dq_empty, it & 1, abort_flag)) break;
+          // The dQ read-out is the one wait on this thread's critical path (the tensor core idles through it), so
+          // it polls without suspending (the dQ warps and the compute warps have slack; measured faster in
+          // paired runs, while spinning on the other waits of this thread was slower).
+          if (!mbar_wait_spin(dq_empty, it & 1, abort_flag)) break;
           tc_fence_after_sync();
           issue_dp(it + 1);
           umma_commit(dp_full);
@@ -455,12 +458,14 @@ __global__ void __launch_bounds__(512, 1)
       // queue of every SM sub-partition, and the MMA thread's tcgen05 instructions, which wait in the same queue,
       // stall behind them (measured, alternating runs on one B200: main kernel 6.26 -> 5.64 ms at
       // 4x32x8192x128, within 4% of a timing copy with no reductions at all). A tile's 64 KB need only ~15 bytes
-      // per cycle of the ~23 an SM sustains.
+      // per cycle of the ~23 an SM sustains. The sleep is bounded from both sides (paired runs): at 20-30 ns
+      // the queues fill again (+18% time), and the 32 sleeps must end well inside one tile's ~5000 cycles, or
+      // the dQ warps become the bottleneck (75 ns: +40%); 50 ns keeps a 20% margin at the top SM clock.
       float* base = p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * (p.Sq_pad / 4) + q0 / 4) * 512 + d * 4;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         red_add_v4(base + static_cast<size_t>(c) * 512, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-        __nanosleep(60);
+        __nanosleep(50);
       }
     }
   }

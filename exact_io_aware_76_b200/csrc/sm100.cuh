@@ -96,6 +96,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_ns(bar, parity, abort_flag, kWaitTimeoutNs);
 }
 
+// Non-blocking test of the phase of parity `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// The same bounded wait, polling with the non-blocking test instead of the potentially suspending try-wait:
+// the thread notices the phase change sooner, at the price of a shared-memory poll every few cycles. Worth it
+// only for a wait that sits on a kernel's critical path while the warps that would feel the polls have slack.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t polls = 1;; ++polls) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((polls & 1023u) == 0u) {
+      if (*abort_flag) return false;
+      if (polls >= kWaitMaxPolls || globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        atomicExch(&g_device_status, FA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------------------------
 // TMA (tiled tensor copies global -> shared, completion counted on an mbarrier). No multicast.
 // ---------------------------------------------------------------------------------------------------------
