@@ -32,6 +32,11 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 NOMINAL_BF16_TFLOPS = 2250.0
+# MUFU (special-function unit) roofline: 16 exponentials per cycle per SM, 148 SMs, at the top SM clock
+# (`clocks.max.sm`, 1965 MHz on these B200s, used when no clock was sampled).
+MUFU_EXP_PER_CYCLE_SM = 16
+N_SMS = 148
+NOMINAL_SM_MHZ = 1965.0
 _COMMON_SOURCES = ["exact_io_aware_76_b200/csrc/sm100.cuh", "exact_io_aware_76_b200/csrc/tmem_ldst.inc",
                    "exact_io_aware_76_b200/csrc/dropout.cuh"]
 KERNEL_SOURCES = {
@@ -503,6 +508,18 @@ def run_ours(args):
         val, ex, desc, threads, _ = oracle_sample(w, q, k, v, do, reps)
         cpu = cpu_baseline_record(w, val, ex, threads, desc)
     clocks = sampler.summary(t_host0, t_host1)
+    # The softmax's exponentials, one per visible (query, key) pair in either kernel, against the MUFU bound; in
+    # tensor-FLOP units that bound is exp/s times the kernel's FLOP per pair (4*D forward, 10*D backward), which
+    # says which of the two units limits the kernel (the forward at head dim 64: MUFU).
+    n_exp = w.B * w.H * w.pairs()
+    mhz = (clocks or {}).get("sm_max_mhz") or NOMINAL_SM_MHZ
+    exp_peak = MUFU_EXP_PER_CYCLE_SM * N_SMS * mhz * 1e6 / 1e9
+    exp_achieved = n_exp / (per_kernel[dom] / 1e3) / 1e9
+    equiv_peak = exp_peak * (dom_flops / n_exp) / 1e3
+    roofline["mufu"] = {"achieved": exp_achieved, "peak": exp_peak, "unit": "Gexp/s", "frac": exp_achieved / exp_peak,
+                        "tflops_equivalent_peak": equiv_peak, "binding": "mufu" if equiv_peak < peak else "tensor",
+                        "peak_source": "%d exp per cycle per SM x %d SMs x %.0f MHz" % (MUFU_EXP_PER_CYCLE_SM, N_SMS,
+                                                                                        mhz)}
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if variant == "fp8" else "bf16", "data": "synthetic",

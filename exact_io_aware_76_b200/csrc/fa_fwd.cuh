@@ -85,8 +85,9 @@ struct FwdSmem {
   // fastest (+5%); with 16-bit inputs any share made the kernel slower, so none.
   static constexpr int kEmuEvery = kFP8 ? 4 : 0;
   // P is handed to the MMA thread in two halves of 64 keys (the first half of PV overlaps the second half of
-  // the exponentials). Measured: +4-6% with 8-bit inputs, -3% with 16-bit ones (one hand-off is cheaper there).
-  static constexpr bool kSplitP = kFP8;
+  // the exponentials). Measured: +4-6% with 8-bit inputs and +3-4% with 16-bit ones at head dim 64 (both have
+  // half the MMA time per tile of 16-bit head dim 128), -3% with 16-bit head dim 128 (one hand-off is cheaper).
+  static constexpr bool kSplitP = kFP8 || D == 64;
 };
 
 // kBF16: the 16-bit input type (and output type); with kFP8 the inputs are e4m3 and the output is bf16.
