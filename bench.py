@@ -153,14 +153,20 @@ class ClockSampler:
             except Exception:
                 return None
 
-        sel = []
+        mine = []
         for (ts, p) in self.rows:
-            if not (t0 <= ts <= t1 + 0.15):
-                continue
             uid = p[1].lower().replace("gpu-", "")
             if self.uuid and uid and uid != self.uuid:
                 continue
-            sel.append(p)
+            mine.append((ts, p))
+        sel = [p for (ts, p) in mine if t0 <= ts <= t1 + 0.15]
+        window = "timed region"
+        if not sel and mine:
+            # A timed region shorter than the sampling period: the samples just before and just after it.
+            before = [(ts, p) for (ts, p) in mine if ts < t0]
+            after = [(ts, p) for (ts, p) in mine if ts > t1]
+            sel = ([before[-1][1]] if before else []) + ([after[0][1]] if after else [])
+            window = "nearest samples before and after the timed region (shorter than the 100 ms sampling period)"
         if not sel:
             return None
         sm = [num(p[2]) for p in sel if num(p[2]) is not None]
@@ -168,7 +174,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for p in sel for i in range(4) if p[6 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(sel),
+                "reasons": reasons, "samples": len(sel), "window": window,
                 "power_w_max": max((num(p[4]) for p in sel if num(p[4]) is not None), default=None)}
 
 
