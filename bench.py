@@ -12,7 +12,10 @@ Prints one JSON line (rank 0). ``value`` is the whole-job TFLOP/s from CUDA even
 in HBM (1.07 GB per step, larger than the 126 MB L2); ``e2e`` is the same metric through the public Python API
 with pinned host inputs copied in and the gradients copied out every step (two buffer sets on separate upload,
 compute and download streams, so step i+1's upload and step i-1's download overlap step i); ``roofline``
-rates the dominant kernel against the measured bf16 peak; ``cpu_baseline`` times the fp64 CPU oracle on a bounded row sample.
+rates the dominant kernel against the measured bf16 peak, and ``roofline.mufu`` its exponentials against the
+MUFU bound (16 per cycle per SM), which binds the head-dim-64 forward; ``clocks`` summarises nvidia-smi samples
+taken in the timed region (or, for a region shorter than the sampling period, the samples on either side);
+``cpu_baseline`` times the fp64 CPU oracle on a bounded row sample.
 With N > 1 (torchrun) every GPU runs its own replica of the workload (weak scaling, no collective on the data
 path) and the time is the maximum over ranks. ``--impl reference`` times the oracle itself as the reference
 arm (rank 0 only).
