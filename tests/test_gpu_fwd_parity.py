@@ -111,6 +111,15 @@ def test_gpt_workload_sampled_rows():
     print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 4, 1)))
 
 
+def test_skill_timing_sampled_rows():
+    """The skill page's timing shape (Workflow 1 Step 4: batch 4, seqlen 4096, 32 heads, head dim 64, fp16, no
+    mask), which runs the head-dim-64 forward with P handed over in two halves; sampled rows of every head."""
+    w = WORKLOADS["skill_timing"]
+    q, k, v = make_workload_inputs(w)
+    hs = all_heads(w.B, w.H)
+    print(run_and_check(q, k, v, w.causal, None, w.sigma, heads=hs, rows=sampled_rows(w.Sq, hs, 6, 3)))
+
+
 def test_long_context_sampled_rows():
     w = WORKLOADS["long"]
     q, k, v = make_workload_inputs(w)
