@@ -212,13 +212,14 @@ int launch_bwd(int stage, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stage < 0 || stage == 1) {
-    const unsigned grid = (unsigned)(p.n_kblk * p.B * p.Hkv);
     if constexpr (D == 128) {
+      const unsigned grid = (unsigned)(p.n_grp * p.B * p.Hkv);
       auto kern = fa::fa_bwd_main128_kernel<BF16, CAUSAL, DROP>;
       int rc = ensure_smem_attr(kern, Bwd128Smem::kAlloc, dev, attr_done);
       if (rc) return rc;
       kern<<<grid, Bwd128Smem::kThreads, Bwd128Smem::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     } else {
+      const unsigned grid = (unsigned)(p.n_kblk * p.B * p.Hkv);
       auto kern = fa::fa_bwd_main_kernel<D, BF16, CAUSAL, DROP>;
       int rc = ensure_smem_attr(kern, BwdSmem<D>::kAlloc, dev, attr_done);
       if (rc) return rc;
@@ -451,6 +452,16 @@ static int bwd_impl(int stage, const void* q, const void* k, const void* v, cons
   p.Sk = Sk;
   p.Sq_pad = lay.sq_pad;
   p.n_kblk = (Sk + 127) / 128;
+  // Head dim 128: several key tiles per CTA when there are enough of them to keep about three waves of CTAs
+  // (a unit's tail then overlaps the next unit's start); one otherwise.
+  p.units = 1;
+  if (D == 128)
+    for (int u : {8, 4, 2})
+      if ((long long)B * Hkv * ((p.n_kblk + u - 1) / u) >= 3LL * g_dev[dev].sm_count) {
+        p.units = u;
+        break;
+      }
+  p.n_grp = (p.n_kblk + p.units - 1) / p.units;
   // Head-major CTA order once Q, dO and the fp32 dQ accumulator no longer fit in L2.
   p.head_major = ((double)B * Sq * H * D * 8 > kHeadMajorBytes) ? 1 : 0;
   p.scale = scale;

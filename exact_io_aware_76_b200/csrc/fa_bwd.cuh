@@ -49,6 +49,7 @@ struct BwdParams {
   int Hkv, group;            // K/V heads and query heads per K/V head (H = Hkv * group)
   int win_left, win_right;   // window around the aligned key i + Sk - Sq; negative = unbounded side
   int n_kblk;        // ceil(Sk / 128)
+  int units, n_grp;  // head dim 128: key tiles per CTA, CTAs per (batch, K/V head) = ceil(n_kblk / units)
   int head_major;    // CTA order: 1 = all key tiles of a head together (L2 reuse), 0 = heavy-first
   float scale, scale_log2;
   uint32_t drop_t;                      // dropout threshold t (0 = no dropout)
