@@ -71,3 +71,26 @@ def test_ex_entry_points_reject_bad_groups():
     L = fa.lib()
     assert L.fa_fwd_ex(p, p, p, p, p, 1, 128, 128, 6, 4, 64, 0, -1, -1, 0.0, 1, None) == -1
     assert L.fa_fwd_ex(p, p, p, p, p, 1, 128, 128, 6, 0, 64, 0, -1, -1, 0.0, 1, None) == -1
+
+
+def test_several_key_tiles_per_cta():
+    """A shape large enough that the head-dim-128 backward gives each CTA two key tiles (32 K/V heads x 48 key
+    tiles), with grouped heads, Sq != Sk and a causal window that leaves the first twelve key tiles without any
+    query, so that CTAs also meet key tiles with nothing to do; dQ/dK/dV of two whole K/V head groups against the
+    oracle, and exact zeros for the keys no query sees."""
+    B, Sq, Sk, H, Hkv, D, window = 1, 4096, 6144, 64, 32, 128, (512, 0)
+    q, k, v, do = make(B, Sq, Sk, H, Hkv, D, "bf16", 6001)
+    out, lse = fa.fwd(q, k, v, causal=True, window=window)
+    dq, dk, dv = fa.bwd(q, k, v, out, lse, do, causal=True, window=window)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    unseen = Sk - Sq - window[0]  # key j is seen by rows r <= j - (Sk - Sq) + left
+    assert dk[:, :unseen].abs().max().item() == 0 and dv[:, :unseen].abs().max().item() == 0
+    assert dk[:, unseen:].abs().max().item() > 0
+    group = H // Hkv
+    for h_kv in (0, Hkv - 1):
+        dq_r, dk_r, dv_r = oracle_bwd_grouped(q, k, v, do, True, None, 0, h_kv, window=window)
+        qh = [(0, h_kv * group + g) for g in range(group)]
+        check_grad(heads_f64(dq, qh), dq_r, "dQ")
+        check_grad(heads_f64(dk, [(0, h_kv)]), dk_r, "dK")
+        check_grad(heads_f64(dv, [(0, h_kv)]), dv_r, "dV")
