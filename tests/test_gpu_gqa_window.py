@@ -74,11 +74,11 @@ def test_ex_entry_points_reject_bad_groups():
 
 
 def test_several_key_tiles_per_cta():
-    """A shape large enough that the head-dim-128 backward gives each CTA two key tiles (32 K/V heads x 48 key
-    tiles), with grouped heads, Sq != Sk and a causal window that leaves the first twelve key tiles without any
-    query, so that CTAs also meet key tiles with nothing to do; dQ/dK/dV of two whole K/V head groups against the
-    oracle, and exact zeros for the keys no query sees."""
-    B, Sq, Sk, H, Hkv, D, window = 1, 4096, 6144, 64, 32, 128, (512, 0)
+    """A shape large enough that the head-dim-128 backward gives each CTA two key tiles (32 K/V heads x 64 key
+    tiles: 1024 CTAs, about seven full waves), with grouped heads, Sq != Sk and a causal window that leaves the
+    first twelve key tiles without any query, so that CTAs also meet key tiles with nothing to do; dQ/dK/dV of
+    two whole K/V head groups against the oracle, and exact zeros for the keys no query sees."""
+    B, Sq, Sk, H, Hkv, D, window = 1, 6144, 8192, 64, 32, 128, (512, 0)
     q, k, v, do = make(B, Sq, Sk, H, Hkv, D, "bf16", 6001)
     out, lse = fa.fwd(q, k, v, causal=True, window=window)
     dq, dk, dv = fa.bwd(q, k, v, out, lse, do, causal=True, window=window)
